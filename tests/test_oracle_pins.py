@@ -1,0 +1,361 @@
+"""Pins of the CPU oracle to what the pages and the mathematics fix (no GPU needed).
+
+Each test names the passage or the closed form it checks. A plausible mistake anywhere in
+the oracle (a wrong digit order, a dropped zero point, double rounding, a transposed
+operand) fails at least one of them; test_planted_mistakes_are_caught shows a few.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import wq_oracle as O
+from bit_weight_quantized_unpack_b200 import workloads
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return [l.rstrip("\n").split() for l in f if l.strip() and not l.startswith("#")]
+
+
+# ---- tables of "The one fact that shapes everything" ----------------------------------
+
+def test_param_table_reproduces_from_layer_shapes():
+    blocks, head, total = O.set_params(workloads.qwen05b_set())
+    assert (blocks, head, total) == (357_826_560, 136_134_656, 493_961_216)
+    gold = {r[0]: r for r in _rows("whetstone_param_table.txt")}
+    assert round(blocks / 1e6, 1) == float(gold["transformer_blocks"][1])
+    assert round(head / 1e6, 1) == float(gold["lm_head"][1])
+    assert round(total / 1e6, 1) == float(gold["total"][1])
+    assert round(100 * blocks / total, 1) == float(gold["transformer_blocks"][2])
+    assert round(100 * head / total, 1) == float(gold["lm_head"][2])
+
+
+def _bpw_closed_form(fmt):
+    # b-bit codes + fp16 scale + fp16 zero per 128 weights; ternary carries log2(3) bits
+    # of information per weight + one fp16 scale per 128; binary 1 bit + one fp16 scale.
+    return {"fp16": 16.0, "int8_per_channel": 8.0, "int4_g128": 4 + 32 / 128,
+            "int3_g128": 3 + 32 / 128, "int2_g128": 2 + 32 / 128,
+            "ternary_g128": math.log2(3) + 16 / 128, "binary_g128": 1 + 16 / 128}[fmt]
+
+
+def test_format_table_reproduces():
+    _, _, total = O.set_params(workloads.qwen05b_set())
+    bw = 278e9
+    checked = 0
+    for fmt, bpw, mb, ceil in _rows("whetstone_format_table.txt"):
+        if fmt == "int4_hier_g32":
+            continue
+        b = _bpw_closed_form(fmt)
+        assert round(b, 2) == float(bpw), fmt
+        mbytes = O.bytes_per_token(total, b) / 1e6
+        assert abs(mbytes - float(mb)) <= 0.05 + 1e-9, (fmt, mbytes, mb)
+        # the page divides by its rounded MB figure; allow the one-unit rounding spread
+        assert abs(O.tok_s_ceiling(bw, float(mb) * 1e6) - float(ceil)) <= 1.0, fmt
+        assert abs(O.tok_s_ceiling(bw, mbytes * 1e6) - float(ceil)) <= 1.0, fmt
+        checked += 1
+    assert checked == 6
+
+
+def test_quality_table_bits_per_weight():
+    for fmt, bpw in _rows("whetstone_quality_bpw.txt"):
+        assert f"{_bpw_closed_form(fmt):.2f}" == bpw, fmt
+
+
+def test_stored_layout_bits_per_weight():
+    assert O.stored_bits_per_weight("int4") == 4.25
+    assert O.stored_bits_per_weight("int2") == 2.25
+    # 26 bytes + one fp16 scale per 128 trits, against the information content 1.71
+    assert O.stored_bits_per_weight("ternary") == 1.75
+    W = np.random.default_rng(0).normal(0, 0.02, (8, 256)).astype(np.float32)
+    for fmt, bits in (("int4", 4.25), ("int2", 2.25), ("ternary", 1.75)):
+        p, s, z = O.quantize(W, fmt)
+        nbytes = p.nbytes + s.nbytes + (0 if z is None else z.nbytes)
+        assert nbytes * 8 / W.size == bits
+
+
+# ---- binary16 rounding routine --------------------------------------------------------
+
+def _parse_val(tok):
+    if tok.startswith("2^"):
+        return 2.0 ** int(tok[2:])
+    if "+" in tok and "^" in tok:           # "1+2^-11" / "1+3*2^-11"
+        a, b = tok.split("+")
+        c, e = (b.split("*") if "*" in b else ("1", b))
+        return float(a) + float(c) * 2.0 ** int(e[2:])
+    if "*" in tok:                           # "3*2^-25"
+        c, e = tok.split("*")
+        return float(c) * 2.0 ** int(e[2:])
+    return float(tok)
+
+
+def test_binary16_textbook_values():
+    for tok, hx in _rows("binary16_values.txt"):
+        v = _parse_val(tok)
+        r = O.f16_round(v)
+        assert int(O.f16_to_bits(r)) == int(hx, 16), tok
+        assert np.array(int(hx, 16), np.uint16).view(np.float16).astype(np.float64) == r
+
+
+def test_binary16_exhaustive_round_trip():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    v = O.f16_from_bits(bits)
+    ref = bits.view(np.float16).astype(np.float64)       # numpy's own decoding
+    fin = np.isfinite(ref)
+    assert np.array_equal(v[fin], ref[fin])
+    assert np.array_equal(np.isnan(v), np.isnan(ref))
+    assert np.array_equal(O.f16_round(v[fin]), v[fin])
+    assert np.array_equal(O.f16_to_bits(v[fin]), bits[fin])
+
+
+def test_binary16_midpoints_ties_to_even_and_neighbours():
+    v = np.sort(np.unique(O.f16_from_bits(np.arange(0, 0x7C00, dtype=np.uint16))))
+    lo, hi = v[:-1], v[1:]
+    mid = (lo + hi) / 2                      # exact in float64
+    even = np.where((O.f16_to_bits(lo) & 1) == 0, lo, hi)
+    assert np.array_equal(O.f16_round(mid), even)
+    assert np.array_equal(O.f16_round(-mid), -even)
+    assert np.array_equal(O.f16_round(np.nextafter(mid, np.inf)), hi)
+    assert np.array_equal(O.f16_round(np.nextafter(mid, -np.inf)), lo)
+
+
+def test_binary16_matches_numpy_direct_conversion():
+    rng = np.random.default_rng(1)
+    d = np.concatenate([rng.normal(0, 1, 200000), rng.normal(0, 1e-5, 100000),
+                        rng.uniform(-7e4, 7e4, 100000)])
+    assert np.array_equal(O.f16_round(d), d.astype(np.float16).astype(np.float64))
+
+
+# ---- quantisers: closed-form cases and properties ------------------------------------
+
+def test_int4_ramp_gives_codes_in_order():
+    # 128 values -1 + 0.125 * (j mod 16): lo = -1, hi = 0.875, s = 1.875 / 15 = 0.125 exactly,
+    # z = rint(1 / 0.125) = 8, q_j = (j mod 16) - 8 + 8.
+    j = np.arange(128)
+    W = (-1 + 0.125 * (j % 16)).reshape(1, 128)
+    codes, s, z = O.quantize_int(W, 4)
+    assert O.f16_from_bits(s)[0, 0] == 0.125 and O.f16_from_bits(z)[0, 0] == 8.0
+    assert np.array_equal(O.unpack_int(codes, 4, 128)[0], j % 16)
+    # word layout: code k at bits 4*(k % 8) of word k // 8 -> word 0 = 0x76543210
+    assert codes[0, 0] == 0x76543210 and codes[0, 1] == 0xFEDCBA98
+
+
+def test_int2_ramp_and_word_layout():
+    j = np.arange(128)
+    W = (0.5 * (j % 4) - 0.5).reshape(1, 128)       # lo -0.5 hi 1.0 -> s 0.5, z 1
+    codes, s, z = O.quantize_int(W, 2)
+    assert O.f16_from_bits(s)[0, 0] == 0.5 and O.f16_from_bits(z)[0, 0] == 1.0
+    assert np.array_equal(O.unpack_int(codes, 2, 128)[0], j % 4)
+    assert codes[0, 0] == 0xE4E4E4E4               # 0,1,2,3 repeating, 2 bits each
+
+
+def test_constant_and_nonnegative_groups():
+    W = np.zeros((2, 256), np.float32)
+    W[1, :128] = 0.25
+    W[1, 128:] = np.linspace(0, 3, 128, dtype=np.float32)      # group in [0, c] -> z = 0
+    codes, s, z = O.quantize_int(W, 4)
+    sv, zv = O.f16_from_bits(s), O.f16_from_bits(z)
+    assert np.all(sv[0] == 1.0) and np.all(zv[0] == 0.0)          # zero range -> s = 1
+    assert np.all(O.dequant_int(codes, s, z, 4, 256)[0] == 0.0)
+    assert sv[1, 0] == 1.0 and zv[1, 0] == 0.0                      # constant 0.25 group
+    assert zv[1, 1] == 0.0 and sv[1, 1] == O.f16_round(3.0 / 15)
+
+
+def test_rtn_is_nearest_code_within_range():
+    rng = np.random.default_rng(2)
+    for bits in (4, 2):
+        Q = 2 ** bits - 1
+        W = rng.normal(0, 0.02, (16, 512)).astype(np.float32)
+        codes, sb, zb = O.quantize_int(W, bits)
+        q = O.unpack_int(codes, bits, 512)
+        s = np.repeat(O.f16_from_bits(sb), 128, axis=1)
+        z = np.repeat(O.f16_from_bits(zb), 128, axis=1)
+        w = W.astype(np.float64)
+        err = np.abs((q - z) * s - w)
+        # brute force over every code: the chosen one is (one of) the nearest
+        best = np.min(np.abs((np.arange(Q + 1)[:, None, None] - z) * s - w), axis=0)
+        assert np.allclose(err, best, rtol=0, atol=1e-15 * np.abs(w).max())
+        inside = (w >= (-z - 0.5) * s) & (w <= (Q - z + 0.5) * s)
+        assert inside.mean() > 0.99 and np.all(err[inside] <= s[inside] / 2 * (1 + 1e-12))
+        assert q.min() >= 0 and q.max() <= Q
+
+
+def test_ternary_closed_forms():
+    a = 0.015625                                    # exactly representable in fp16
+    sign = np.where(np.arange(128) % 3 == 0, -1.0, 1.0)
+    W = np.stack([a * sign, np.zeros(128), np.r_[np.full(64, 0.5), np.zeros(64)]])
+    p, s = O.quantize_ternary(W.astype(np.float32))
+    sv = O.f16_from_bits(s)[:, 0]
+    t = O.unpack_ternary(p, 128)
+    assert sv[0] == a and np.array_equal(t[0], sign.astype(int))
+    assert sv[1] == 1.0 and np.all(t[1] == 0)                      # zero group -> s = 1
+    # absmean 0.25: values 0.5 -> rint(2) clamps to 1, zeros stay 0
+    assert sv[2] == 0.25 and np.all(t[2, :64] == 1) and np.all(t[2, 64:] == 0)
+    assert p.shape == (3, 26) and p[1, 25] == 121                  # pads are trit 0
+
+
+def test_ternary_absmean_is_sequential_float64_sum():
+    # 1.0 then 127 copies of 2^-53: float64 sequential sum keeps 1.0 at every step.
+    W = np.r_[1.0, np.full(127, 2.0 ** -53)].astype(np.float32).reshape(1, 128)
+    _, s = O.quantize_ternary(W)
+    assert O.f16_from_bits(s)[0, 0] == O.f16_round(1.0 / 128)
+
+
+# ---- base-3 codec --------------------------------------------------------------------
+
+def test_base3_golden_bytes():
+    for r in _rows("base3_bytes.txt"):
+        t5, b = tuple(int(v) for v in r[:5]), int(r[5])
+        assert O.trits_to_byte(t5) == b
+        assert O.byte_to_trits(b) == t5
+
+
+def test_base3_exhaustive_243_round_trip():
+    seen = set()
+    for b in range(243):
+        t5 = O.byte_to_trits(b)
+        assert all(t in (-1, 0, 1) for t in t5)
+        assert O.trits_to_byte(t5) == b
+        assert sum(t * 3 ** i for i, t in enumerate(t5)) + 121 == b
+        seen.add(t5)
+    assert len(seen) == 243
+    for b in range(243, 256):
+        with pytest.raises(ValueError):
+            O.byte_to_trits(b)
+    bad = np.full((1, 26), 243, np.uint8)
+    with pytest.raises(ValueError):
+        O.unpack_ternary(bad, 128)
+
+
+def test_ternary_pack_matches_scalar_codec():
+    rng = np.random.default_rng(3)
+    t = rng.integers(-1, 2, (4, 256))
+    p = O.pack_ternary(t)
+    assert p.shape == (4, 52)
+    for n in range(4):
+        for g in range(2):
+            grp = list(t[n, 128 * g:128 * (g + 1)]) + [0, 0]
+            for j in range(26):
+                assert p[n, 26 * g + j] == O.trits_to_byte(tuple(grp[5 * j:5 * j + 5]))
+    assert np.array_equal(O.unpack_ternary(p, 256), t)
+
+
+# ---- the +-1 identity ----------------------------------------------------------------
+
+def test_pm1_identity_brute_force():
+    for K in range(1, 11):
+        vals = np.array([[1 if (a >> i) & 1 else -1 for i in range(K)] for a in range(2 ** K)])
+        dots = vals @ vals.T
+        for a in range(2 ** K):
+            for b in range(2 ** K):
+                assert O.pm1_dot_popcount(a, b, K) == dots[a, b]
+
+
+def test_ternary_unpack_through_pm1_identity():
+    # every base-3 code, decoded, dotted with every +-1 vector of length 5
+    for byte in range(243):
+        t5 = O.byte_to_trits(byte)
+        for a in range(32):
+            av = [1 if (a >> i) & 1 else -1 for i in range(5)]
+            assert O.ternary_pm1_dot_popcount(a, t5) == sum(x * t for x, t in zip(av, t5))
+    # a packed group, unpacked, against the identity on its +-1 weights
+    rng = np.random.default_rng(4)
+    t = rng.integers(-1, 2, (1, 128))
+    tt = O.unpack_ternary(O.pack_ternary(t), 128)[0]
+    a = int(rng.integers(0, 2 ** 62)) | (int(rng.integers(0, 2 ** 62)) << 62)
+    av = np.array([1 if (a >> i) & 1 else -1 for i in range(128)])
+    assert O.ternary_pm1_dot_popcount(a, list(tt)) == int(av @ t[0])
+
+
+# ---- the product ---------------------------------------------------------------------
+
+def test_linear_matches_exact_rational_sum():
+    rng = np.random.default_rng(5)
+    W = rng.normal(0, 0.02, (3, 256)).astype(np.float32)
+    x = rng.normal(0, 1, (2, 256)).astype(np.float16)
+    for fmt in ("int4", "int2", "ternary"):
+        p, s, z = O.quantize(W, fmt)
+        y, bound = O.gemv_packed(x, fmt, p, s, z, 256)
+        w_hat = (O.dequant_ternary(p, s, 256) if fmt == "ternary"
+                 else O.dequant_int(p, s, z, {"int4": 4, "int2": 2}[fmt], 256))
+        for m in range(2):
+            for n in range(3):
+                exact = sum(Fraction(float(x[m, k])) * Fraction(w_hat[n, k]) for k in range(256))
+                babs = sum(abs(Fraction(float(x[m, k])) * Fraction(w_hat[n, k])) for k in range(256))
+                assert abs(Fraction(y[m, n]) - exact) <= Fraction(1, 10 ** 12) * babs
+                assert abs(Fraction(bound[m, n]) - babs) <= Fraction(1, 10 ** 12) * babs
+
+
+def test_dequant_matches_scalar_definition():
+    rng = np.random.default_rng(6)
+    W = rng.normal(0, 0.02, (2, 256)).astype(np.float32)
+    codes, sb, zb = O.quantize_int(W, 4)
+    w_hat = O.dequant_int(codes, sb, zb, 4, 256)
+    for n in range(2):
+        for k in range(0, 256, 7):
+            word = int(codes[n, k // 8])
+            q = (word >> (4 * (k % 8))) & 0xF
+            s = float(np.array(sb[n, k // 128]).view(np.float16))
+            z = float(np.array(zb[n, k // 128]).view(np.float16))
+            assert w_hat[n, k] == (q - z) * s
+
+
+def test_linear_special_cases():
+    rng = np.random.default_rng(7)
+    W = rng.normal(0, 0.02, (5, 256)).astype(np.float32)
+    codes, sb, zb = O.quantize_int(W, 4)
+    # all codes equal to the zero point -> y = 0 exactly
+    q = np.repeat(O.f16_from_bits(zb), 128, axis=1).astype(np.int64)
+    codes0 = O.pack_int(q, 4)
+    x = rng.normal(0, 1, 256).astype(np.float16)
+    y0, _ = O.gemv_packed(x, "int4", codes0, sb, zb, 256)
+    assert np.all(y0 == 0.0)
+    # x = e_k picks column k of w_hat
+    w_hat = O.dequant_int(codes, sb, zb, 4, 256)
+    for k in (0, 127, 128, 255):
+        e = np.zeros(256, np.float16)
+        e[k] = 1
+        y, _ = O.gemv_packed(e, "int4", codes, sb, zb, 256)
+        assert np.array_equal(y, w_hat[:, k])
+    # batched rows equal separate vectors (no transposed operand)
+    X = rng.normal(0, 1, (3, 256)).astype(np.float16)
+    Y, _ = O.gemv_packed(X, "int4", codes, sb, zb, 256)
+    for m in range(3):
+        ym, _ = O.gemv_packed(X[m], "int4", codes, sb, zb, 256)
+        assert np.allclose(Y[m], ym, rtol=1e-14, atol=0)
+    assert Y.shape == (3, 5)
+
+
+# ---- planted mistakes are caught -----------------------------------------------------
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    j = np.arange(128)
+    ramp = (-1 + 0.125 * (j % 16)).reshape(1, 128)
+
+    # (a) zero point dropped from the code
+    def q_no_zero(W, bits):
+        N, K = W.shape
+        w = W.astype(np.float64).reshape(N, K // 128, 128)
+        lo, hi = w.min(2), w.max(2)
+        s = O.f16_round((hi - lo) / 15)
+        q = np.clip(np.rint(w / s[:, :, None]), 0, 15).astype(np.uint32)
+        return O.pack_int(q.reshape(N, K), bits), O.f16_to_bits(s), O.f16_to_bits(0 * s)
+    codes, _, _ = q_no_zero(ramp, 4)
+    assert not np.array_equal(O.unpack_int(codes, 4, 128)[0], j % 16)
+
+    # (b) base-3 digits in the opposite order
+    def rev(t5):
+        return sum((int(t) + 1) * 3 ** (4 - i) for i, t in enumerate(t5))
+    assert any(rev(tuple(int(v) for v in r[:5])) != int(r[5]) for r in _rows("base3_bytes.txt"))
+
+    # (c) float64 -> float32 -> float16 double rounding
+    d = 1 + 2.0 ** -11 + 2.0 ** -40          # just above a binary16 midpoint
+    assert np.float16(np.float32(d)) != O.f16_round(d)
+
+    # (d) identity with a wrong factor
+    assert any((K - bin(a ^ b).count("1")) != O.pm1_dot_popcount(a, b, K)
+               for K in (3,) for a in range(8) for b in range(8))
