@@ -1,0 +1,396 @@
+"""Benchmark: int4 g128 batch-1 GEMV weight GB/s on the Qwen2.5-0.5B-shaped decode set.
+
+One step = one decoded token's worth of linear layers: all 169 matrices of the set
+(24 layers x q, k, v, o, gate, up, down + the 151936-row lm_head, 493,961,216 int4 g128
+weights = 262.42 MB of codes + scales + zeros) in one wq_linear_set launch. `value` is
+weight bytes per second with everything resident in HBM; `e2e` is the same through the
+public API with the activations copied in from pinned host memory and the outputs
+copied back inside the timed region. Secondary rows (lm_head formats, quantiser,
+batch sweep, M=512 prefill GEMM) are reported under "rows".
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+Under torchrun (N > 1) every rank runs an independent replica on its own GPU (the
+decode set has no data-path exchange); rank 0 prints the JSON line with the
+max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_weight_quantized_unpack_b200 import synth, workloads  # noqa: E402
+
+METRIC = "int4 g128 batch-1 GEMV weight GB/s (% of HBM peak); M=512 GEMM TFLOPS"
+INT4_BYTES_PER_WEIGHT = 0.5 + 4 / 128  # codes + fp16 scale + fp16 zero per 128 weights
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, ws
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, ws):
+    if ws == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            idx = str(torch.cuda.current_device())
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                idx = vis.split(",")[torch.cuda.current_device()]
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", idx, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+
+def build_set(widx, copies, fmt="int4"):
+    """Quantise `copies` independent copies of a workload's layer set on the GPU."""
+    from bit_weight_quantized_unpack_b200 import wq
+    wl = workloads.WORKLOADS[widx]
+    mats = workloads.workload_mats(widx)
+    K_tot = sum(m.K for m in mats)
+    N_tot = sum(m.N for m in mats)
+    sets = []
+    for cidx in range(copies):
+        x_all = torch.empty(K_tot, dtype=torch.float16, device="cuda")
+        y_all = torch.empty(N_tot, dtype=torch.float16, device="cuda")
+        ent, ko, no = [], 0, 0
+        for i, m in enumerate(mats):
+            seed = synth.sub_seed(wl["seed"] + 7919 * cidx, i, 0)
+            W = synth.weights(m.N, m.K, wl["sigma"], seed, device="cuda")
+            c, s, z = wq.alloc_packed(m.N, m.K, fmt)
+            wq.wq_quantize(W, m.N, m.K, fmt, 128, c, s, z)
+            del W
+            x = x_all[ko:ko + m.K]
+            x.copy_(synth.activations(1, m.K, synth.sub_seed(wl["seed"], i, 1), device="cuda")[0])
+            ent.append((c, s, z, x, y_all[no:no + m.N], m.N, m.K))
+            ko += m.K
+            no += m.N
+        sets.append({"desc": wq.make_linear_set(ent), "count": len(ent), "ent": ent,
+                     "x_all": x_all, "y_all": y_all})
+    torch.cuda.synchronize()
+    weights = sum(m.N * m.K for m in mats)
+    return sets, weights, K_tot, N_tot
+
+
+def time_steps(step, steps, warmup, ws, clocks=None):
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx = clocks if clocks is not None else _Null()
+    with ctx:
+        torch.cuda.synchronize()
+        ev0.record()
+        for i in range(steps):
+            step(i)
+        ev1.record()
+        torch.cuda.synchronize()
+    barrier(ws)
+    return ev0.elapsed_time(ev1) / steps  # ms per step on this rank
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        pass
+
+
+def bench_rows(args, pk):
+    """Secondary measurements of the other hot-path rows (1 GPU)."""
+    from bit_weight_quantized_unpack_b200 import wq
+    rows = {}
+    N, K = 151936, 896
+    wl = workloads.WORKLOADS[2]
+    # lm_head alone, each format; 4+ rotating copies so the working set exceeds L2
+    for fmt in ("int4", "int2", "ternary"):
+        copies = []
+        for cidx in range(6 if fmt != "int4" else 4):
+            W = synth.weights_with_outliers(N, K, wl["sigma"], synth.sub_seed(wl["seed"] + cidx, 0, 0),
+                                            wl["outlier_frac"], wl["outlier_gain"], device="cuda")
+            c, s, z = wq.alloc_packed(N, K, fmt)
+            if fmt == "int4" and cidx == 0:
+                # quantiser throughput (row a1/a2 measured on the int4 path)
+                ev0, ev1 = torch.cuda.Event(True), torch.cuda.Event(True)
+                wq.wq_quantize(W, N, K, fmt, 128, c, s, z)
+                ev0.record()
+                for _ in range(5):
+                    wq.wq_quantize(W, N, K, fmt, 128, c, s, z)
+                ev1.record()
+                torch.cuda.synchronize()
+                ms = ev0.elapsed_time(ev1) / 5
+                rows["quantize_int4_lm_head"] = {"ms": ms, "W_GBps": N * K * 4 / ms / 1e6}
+            wq.wq_quantize(W, N, K, fmt, 128, c, s, z)
+            del W
+            copies.append((c, s, z))
+        x = synth.activations(1, K, 99, device="cuda")[0]
+        y = torch.empty(N, dtype=torch.float16, device="cuda")
+        nb = wq.wq_codes_bytes(fmt, N, K) + 2 * wq.wq_meta_count(N, K) * (1 if fmt == "ternary" else 2)
+
+        def step(i, copies=copies, fmt=fmt):
+            c, s, z = copies[i % len(copies)]
+            wq.wq_gemv(x, c, s, z, fmt, N, K, y)
+        ms = time_steps(step, 200 if not args.quick else 20, 10, 1)
+        rows[f"gemv_lm_head_{fmt}"] = {"ms": ms, "GBps": nb / ms / 1e6,
+                                       "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"]}
+        del copies
+        torch.cuda.empty_cache()
+    return rows
+
+
+def run_ours(args):
+    rank, ws = dist_init()
+    torch.cuda.init()
+    from bit_weight_quantized_unpack_b200 import wq
+    pk = peaks()
+    sets, weights, K_tot, N_tot = build_set(1, copies=2)
+    nbytes = weights * INT4_BYTES_PER_WEIGHT
+
+    def step(i):
+        s = sets[i % len(sets)]
+        wq.wq_linear_set(s["desc"], s["count"], "int4")
+
+    clocks = Clocks()
+    ms = time_steps(step, args.steps, args.warmup, ws, clocks)
+    ms_max = max_over_ranks(ms, ws)
+    gbs = nbytes / ms_max / 1e6 * ws  # whole job: every rank processed one set per step
+
+    # e2e: pinned host activations in, outputs out, inside the timed region
+    x_host = torch.empty(K_tot, dtype=torch.float16, pin_memory=True)
+    x_host.copy_(sets[0]["x_all"].cpu())
+    y_host = torch.empty(N_tot, dtype=torch.float16, pin_memory=True)
+
+    def step_e2e(i):
+        s = sets[i % len(sets)]
+        s["x_all"].copy_(x_host, non_blocking=True)
+        wq.wq_linear_set(s["desc"], s["count"], "int4")
+        y_host.copy_(s["y_all"], non_blocking=True)
+
+    e2e_steps = max(args.steps // 4, 10)
+    ms_e2e = max_over_ranks(time_steps(step_e2e, e2e_steps, args.warmup, ws), ws)
+
+    rows = bench_rows(args, pk) if (rank == 0 and ws == 1 and not args.no_rows) else {}
+
+    if rank == 0:
+        cpu = cpu_baseline(args) if ws == 1 else None
+        line = {
+            "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16 x int4 -> f32", "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1) fp16 x)",
+            "config": {"workload": workloads.WORKLOADS[1]["name"], "matrices": len(sets[0]["ent"]),
+                       "weights": weights, "weight_bytes_per_step": nbytes, "batch": 1,
+                       "launch": "one wq_linear_set (persistent) per step",
+                       "l2": "inputs larger than L2: 2 rotating copies of the set (525 MB)",
+                       "parallelism": f"replicas x{ws}"},
+            "implied_tok_s": round(1e3 / ms_max, 1),
+            "frac_of_hbm_peak": round(gbs / ws / pk["hbm_gbs"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(nbytes / ms / 1e6, 2),
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(nbytes / ms / 1e6 / pk["hbm_gbs"], 4),
+                         "traffic": None, "kernel": "gemv_int_set_kernel<4,1>",
+                         "peak_source": pk["source"]},
+            "e2e": {"value": round(nbytes * ws / ms_e2e / 1e6, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": 2 * K_tot, "d2h_bytes_per_step": 2 * N_tot},
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+            "rows": rows,
+        }
+        print(json.dumps(line), flush=True)
+    barrier(ws)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------------
+# oracle arms (host cores)
+# ---------------------------------------------------------------------------------------
+
+def _oracle_sample(rows_div=64):
+    """A bounded sample of the decode set: every rows_div-th row of every matrix, with the
+    oracle's own quantisation done before timing. Returns (list of (x, packed...), weights)."""
+    import numpy as np
+    from oracle import wq_oracle as O
+    wl = workloads.WORKLOADS[1]
+    sample, weights = [], 0
+    for i, m in enumerate(workloads.workload_mats(1)):
+        n = max(1, m.N // rows_div)
+        W = synth.weights(n, m.K, wl["sigma"], synth.sub_seed(wl["seed"], i, 0) ^ 0xC0FFEE)
+        x = synth.activations(1, m.K, synth.sub_seed(wl["seed"], i, 1))[0].numpy()
+        sample.append((x, O.quantize(W.numpy(), "int4"), m.K))
+        weights += n * m.K
+    return sample, weights
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(args):
+    from oracle import wq_oracle as O
+    sample, weights = _oracle_sample(256 if args.quick else 64)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for x, (p, s, z), K in sample:
+            O.gemv_packed(x, "int4", p, s, z, K)
+        reps += 1
+        if time.perf_counter() - t0 > (2.0 if args.quick else 10.0):
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(weights * INT4_BYTES_PER_WEIGHT / dt / 1e9, 4), "unit": "GB/s",
+            "cores": _threads(), "kind": "oracle",
+            "sample": f"every {256 if args.quick else 64}th row of each of the 169 matrices "
+                      f"({weights} weights), dequantise + float64 product, {reps} reps"}
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import wq_oracle as O
+    # size each step's sample so that warmup + steps take about 90 s of host time
+    cal, cal_w = _oracle_sample(1024)
+    t0 = time.perf_counter()
+    for x, (p, s, z), K in cal:
+        O.gemv_packed(x, "int4", p, s, z, K)
+    t_cal = time.perf_counter() - t0
+    budget = 90.0 / (args.steps + args.warmup)
+    rows_div = int(min(max(1024 * t_cal / budget, 64), 1 << 20))
+    sample, weights = _oracle_sample(rows_div)
+    nbytes = weights * INT4_BYTES_PER_WEIGHT
+
+    def step():
+        for x, (p, s, z), K in sample:
+            O.gemv_packed(x, "int4", p, s, z, K)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = round(nbytes / dt / 1e9, 4)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workloads.WORKLOADS[1]["name"],
+                                            "sample": f"every {rows_div}th row of each matrix"},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+                             "sample": f"every {rows_div}th row of each of the 169 matrices "
+                                       f"({weights} weights)"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--quick", action="store_true", help="smaller rows / CPU sample")
+    ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,138 @@
+// Group-128 quantisers (int4 / int2 asymmetric round-to-nearest, ternary absmean).
+//
+// Whetstone README, "What the weights can actually survive": round-to-nearest with group
+// 128 and one fp16 scale plus one fp16 zero per group (format table rows "int4 g128",
+// "int2 g128"), and a ternary g128 row; TKintegers K5, "What is K5?": five trits per byte.
+// The arithmetic is float64 with correctly rounded division, rint (ties to even) and a
+// direct float64 -> binary16 conversion, so that the codes and metadata are bit-identical
+// to the float64 definition in wq.h. This file is compiled with --fmad=false: no
+// expression may be contracted into a fused multiply-add.
+//
+// Data layout: one warp per (row, group). Lane l reads w[4l .. 4l+3] of the group (one
+// coalesced 512-byte read per warp) and produces those four codes.
+#include "common.cuh"
+
+namespace wq {
+
+__device__ __forceinline__ uint16_t f64_to_f16_bits(double v) {
+  return __half_as_ushort(__double2half(v));  // cvt.rn.f16.f64: one rounding, ties to even
+}
+__device__ __forceinline__ double f16_bits_to_f64(uint16_t b) {
+  return (double)__half2float(__ushort_as_half(b));  // exact widening
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(256) quantize_int_kernel(const float* __restrict__ W, int64_t N,
+                                                           int64_t K, uint32_t* __restrict__ codes,
+                                                           uint16_t* __restrict__ scale,
+                                                           uint16_t* __restrict__ zero) {
+  const int lane = threadIdx.x & 31;
+  const int64_t G = K / kGroup;
+  const int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (task >= N * G) return;
+  const int64_t n = task / G, g = task - n * G;
+
+  const float4 v = *reinterpret_cast<const float4*>(W + n * K + g * kGroup + 4 * lane);
+  float lo = fminf(fminf(v.x, v.y), fminf(v.z, v.w));
+  float hi = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  constexpr double Q = (double)((1 << BITS) - 1);
+  const double dlo = (double)lo, dhi = (double)hi;
+  uint16_t s_bits = f64_to_f16_bits((dhi - dlo) / Q);
+  double s = f16_bits_to_f64(s_bits);
+  if (s == 0.0) {
+    s = 1.0;
+    s_bits = 0x3C00;
+  }
+  const double z = fmin(fmax(rint(-dlo / s), 0.0), Q);
+
+  const float wv[4] = {v.x, v.y, v.z, v.w};
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double q = fmin(fmax(rint((double)wv[i] / s) + z, 0.0), Q);
+    packed |= (uint32_t)q << (BITS * i);
+  }
+  if (BITS == 4) {
+    // lanes 2j and 2j+1 hold codes 8j..8j+3 and 8j+4..8j+7 of word j
+    packed <<= 16 * (lane & 1);
+    packed |= __shfl_xor_sync(0xffffffffu, packed, 1);
+    if ((lane & 1) == 0) codes[n * (K / 8) + g * 16 + (lane >> 1)] = packed;
+  } else {
+    // lanes 4j..4j+3 hold codes 16j..16j+15 of word j, 4 codes (8 bits) each
+    packed <<= 8 * (lane & 3);
+    packed |= __shfl_xor_sync(0xffffffffu, packed, 1);
+    packed |= __shfl_xor_sync(0xffffffffu, packed, 2);
+    if ((lane & 3) == 0) codes[n * (K / 16) + g * 8 + (lane >> 2)] = packed;
+  }
+  if (lane == 0) {
+    scale[task] = s_bits;
+    zero[task] = f64_to_f16_bits(z) & 0x7FFFu;  // small integer: exact; no negative zero
+  }
+}
+
+__global__ void __launch_bounds__(256) quantize_ternary_kernel(const float* __restrict__ W,
+                                                               int64_t N, int64_t K,
+                                                               uint8_t* __restrict__ packed,
+                                                               uint16_t* __restrict__ scale) {
+  __shared__ float s_abs[8][kGroup];
+  __shared__ uint8_t s_dig[8][kTernaryGroupBytes * 5];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t G = K / kGroup;
+  const int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + wid;
+  if (task >= N * G) return;  // whole warps exit together: task is warp-uniform
+  const int64_t n = task / G, g = task - n * G;
+
+  const float4 v = *reinterpret_cast<const float4*>(W + n * K + g * kGroup + 4 * lane);
+  const float wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) s_abs[wid][4 * lane + i] = fabsf(wv[i]);
+  __syncwarp();
+  // absmean: the float64 sum is taken strictly left to right (its rounding depends on
+  // the order), so one lane does it; the group is 128 adds and this kernel is offline.
+  double a = 0.0;
+  if (lane == 0) {
+    for (int k = 0; k < kGroup; ++k) a = __dadd_rn(a, (double)s_abs[wid][k]);
+  }
+  a = __shfl_sync(0xffffffffu, a, 0);
+  uint16_t s_bits = f64_to_f16_bits(a / (double)kGroup);
+  double s = f16_bits_to_f64(s_bits);
+  if (s == 0.0) {
+    s = 1.0;
+    s_bits = 0x3C00;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double t = fmin(fmax(rint((double)wv[i] / s), -1.0), 1.0);
+    s_dig[wid][4 * lane + i] = (uint8_t)(int)(t + 1.0);  // base-3 digit 0, 1, 2
+  }
+  if (lane < 2) s_dig[wid][kGroup + lane] = 1;  // two pad trits of value 0
+  __syncwarp();
+  if (lane < kTernaryGroupBytes) {
+    const uint8_t* d = &s_dig[wid][5 * lane];
+    const uint32_t byte = d[0] + 3u * d[1] + 9u * d[2] + 27u * d[3] + 81u * d[4];
+    packed[n * (kTernaryGroupBytes * G) + g * kTernaryGroupBytes + lane] = (uint8_t)byte;
+  }
+  if (lane == 0) scale[task] = s_bits;
+}
+
+cudaError_t launch_quantize(const float* W, int64_t N, int64_t K, int fmt, void* codes,
+                            uint16_t* scale, uint16_t* zero, cudaStream_t stream) {
+  const int64_t tasks = N * (K / kGroup);
+  const int64_t blocks = (tasks + 7) / 8;
+  if (fmt == 0)
+    quantize_int_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(W, N, K, (uint32_t*)codes, scale,
+                                                                 zero);
+  else if (fmt == 1)
+    quantize_int_kernel<2><<<(unsigned)blocks, 256, 0, stream>>>(W, N, K, (uint32_t*)codes, scale,
+                                                                 zero);
+  else
+    quantize_ternary_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, N, K, (uint8_t*)codes, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace wq

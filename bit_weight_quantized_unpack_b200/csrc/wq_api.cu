@@ -1,0 +1,167 @@
+// C ABI of libwq (declared in include/wq.h): argument checks, launch planning, launches.
+// Every check happens before the first launch; no device memory is ever allocated here.
+#include <limits.h>
+#include <string.h>
+
+#include "gemv.cuh"
+#include "wq.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return WQ_OK;
+  g_last_cuda_error = (int)e;
+  return WQ_ERR_CUDA;
+}
+
+// The kernels are built for sm_100a only: refuse any other device up front instead of
+// failing inside a launch. Cached per device ordinal.
+int check_device() {
+  static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= 64) return WQ_ERR_UNSUPPORTED;
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cached[dev] == 1 ? WQ_OK : WQ_ERR_UNSUPPORTED;
+}
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+constexpr int64_t kMaxK = (int64_t)1 << 20;
+
+int check_shape(int fmt, int64_t N, int64_t K) {
+  if (fmt < WQ_INT4 || fmt > WQ_TERNARY) return WQ_ERR_ARG;
+  if (N < 1 || N > INT_MAX || K < 128 || K > kMaxK || K % 128 != 0) return WQ_ERR_SHAPE;
+  return WQ_OK;
+}
+
+int check_weights(int fmt, const void* codes, const uint16_t* scale, const uint16_t* zero) {
+  if (!codes || !scale) return WQ_ERR_ARG;
+  if ((fmt == WQ_TERNARY) != (zero == nullptr)) return WQ_ERR_ARG;
+  if (!aligned(codes, 16) || !aligned(scale, 2) || (zero && !aligned(zero, 2))) return WQ_ERR_ALIGN;
+  return WQ_OK;
+}
+
+// Fill one SetMat; returns its item count (rows per item = 32 >> lanes_log2).
+int64_t plan_mat(wq::SetMat& m, int fmt, const void* codes, const uint16_t* scale,
+                 const uint16_t* zero, const uint16_t* x, uint16_t* y, int64_t N, int64_t K,
+                 int64_t M) {
+  m.codes = codes;
+  m.scale = scale;
+  m.zero = zero;
+  m.x = x;
+  m.y = y;
+  m.N = (int)N;
+  m.K = (int)K;
+  m.M = (int)M;
+  m.ldx = (int)K;
+  m.ldy = (int)N;
+  m.lanes_log2 = wq::gemv_lanes_log2(fmt, K);
+  const int64_t rows = 32 >> m.lanes_log2;
+  return (N + rows - 1) / rows;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t wq_codes_bytes(int fmt, int64_t N, int64_t K) {
+  if (check_shape(fmt, N, K) != WQ_OK) return 0;
+  if (fmt == WQ_INT4) return (size_t)(N * K / 2);
+  if (fmt == WQ_INT2) return (size_t)(N * K / 4);
+  return (size_t)(N * 26 * (K / 128));
+}
+
+size_t wq_meta_count(int64_t N, int64_t K) {
+  if (check_shape(WQ_INT4, N, K) != WQ_OK) return 0;
+  return (size_t)(N * (K / 128));
+}
+
+int wq_quantize(const float* W, int64_t N, int64_t K, int fmt, int group, void* codes,
+                uint16_t* scale, uint16_t* zero, void* stream) {
+  int st = check_shape(fmt, N, K);
+  if (st != WQ_OK) return st;
+  if (group != 128 || !W) return WQ_ERR_ARG;
+  if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
+  if (!aligned(W, 16)) return WQ_ERR_ALIGN;
+  if ((st = check_device()) != WQ_OK) return st;
+  return cuda_status(wq::launch_quantize(W, N, K, fmt, codes, scale, zero, (cudaStream_t)stream));
+}
+
+int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* scale,
+            const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* Y, void* stream) {
+  int st = check_shape(fmt, N, K);
+  if (st != WQ_OK) return st;
+  if (M < 1 || M > 2048) return WQ_ERR_SHAPE;
+  if (!X || !Y) return WQ_ERR_ARG;
+  if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
+  if (!aligned(X, 16) || !aligned(Y, 2)) return WQ_ERR_ALIGN;
+  if ((st = check_device()) != WQ_OK) return st;
+  wq::SetParams p;
+  p.count = 1;
+  const int64_t items = plan_mat(p.m[0], fmt, codes, scale, zero, X, Y, N, K, M);
+  p.m[0].item_begin = 0;
+  p.m[0].item_end = (int)items;
+  p.total_items = (int)items;
+  return cuda_status(wq::launch_gemv_set(p, fmt, (int)M, (cudaStream_t)stream));
+}
+
+int wq_gemv(const uint16_t* x, const void* codes, const uint16_t* scale, const uint16_t* zero,
+            int fmt, int64_t N, int64_t K, uint16_t* y, void* stream) {
+  return wq_gemm(x, 1, codes, scale, zero, fmt, N, K, y, stream);
+}
+
+int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream) {
+  if (!descs || count < 1 || count > WQ_LINEAR_SET_MAX) return WQ_ERR_ARG;
+  if (fmt < WQ_INT4 || fmt > WQ_TERNARY) return WQ_ERR_ARG;
+  static_assert(WQ_LINEAR_SET_MAX == wq::kSetMax, "set size");
+  wq::SetParams p;
+  p.count = count;
+  int64_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    const wq_linear_desc& d = descs[i];
+    int st = check_shape(fmt, d.N, d.K);
+    if (st != WQ_OK) return st;
+    if (!d.x || !d.y) return WQ_ERR_ARG;
+    if ((st = check_weights(fmt, d.codes, d.scale, d.zero)) != WQ_OK) return st;
+    if (!aligned(d.x, 16) || !aligned(d.y, 2)) return WQ_ERR_ALIGN;
+    const int64_t items = plan_mat(p.m[i], fmt, d.codes, d.scale, d.zero, d.x, d.y, d.N, d.K, 1);
+    p.m[i].item_begin = (int)total;
+    total += items;
+    if (total > INT_MAX) return WQ_ERR_SHAPE;
+    p.m[i].item_end = (int)total;
+  }
+  for (int i = count; i < wq::kSetMax; ++i) {
+    memset(&p.m[i], 0, sizeof(p.m[i]));
+    p.m[i].item_begin = p.m[i].item_end = (int)total;
+  }
+  p.total_items = (int)total;
+  int st = check_device();
+  if (st != WQ_OK) return st;
+  return cuda_status(wq::launch_gemv_set(p, fmt, 1, (cudaStream_t)stream));
+}
+
+const char* wq_status_str(int status) {
+  switch (status) {
+    case WQ_OK: return "WQ_OK";
+    case WQ_ERR_ARG: return "WQ_ERR_ARG: invalid argument (null pointer, format or group)";
+    case WQ_ERR_SHAPE: return "WQ_ERR_SHAPE: N, K or M outside the supported range";
+    case WQ_ERR_ALIGN: return "WQ_ERR_ALIGN: pointer not aligned as required";
+    case WQ_ERR_CUDA: return "WQ_ERR_CUDA: a CUDA call or launch failed";
+    case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+    default: return "unknown wq_status";
+  }
+}
+
+int wq_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

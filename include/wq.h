@@ -1,0 +1,136 @@
+/*
+ * wq.h -- C ABI of libwq: group-quantised sub-byte weights times fp16 activations, on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  A linear layer y = x . W^T whose weight W [N, K] (N output rows, K
+ * along the reduction) is stored quantised in groups of 128 consecutive k of one row:
+ *   - WQ_INT4 / WQ_INT2: asymmetric round-to-nearest b-bit codes q in [0, 2^b - 1] with
+ *     one fp16 scale s and one fp16 integer zero point z per group, w_hat = (q - z) * s
+ *     (Whetstone README, "What the weights can actually survive": round-to-nearest,
+ *     group 128, fp16 scale and zero per group; format table rows "int4 g128" 4.25 and
+ *     "int2 g128" 2.25 bits/weight);
+ *   - WQ_TERNARY: trits t in {-1, 0, +1} with one fp16 absmean scale per group,
+ *     w_hat = t * s, five trits per byte in base 3 (format table row "ternary g128";
+ *     TKintegers K5, "What is K5?": five balanced-ternary digits make a one-byte code).
+ * Products accumulate in fp32; y is rounded to fp16 once, to nearest-even.
+ * Batch-1 decode is bound by memory bandwidth (Whetstone README, "The one fact that
+ * shapes everything": tok/s ceiling = bandwidth / bytes read per token), so the
+ * matrix-vector kernels stream the packed codes once and never materialise w_hat.
+ *
+ * Quantiser definition (bit-exact between the GPU and the float64 reference), per
+ * (row, group), all in float64 with correctly rounded division and rint = ties-to-even:
+ *   int-b:   lo = min w, hi = max w, Q = 2^b - 1
+ *            s = fp16_rne((hi - lo) / Q), s := 1 if s == 0
+ *            z = clamp(rint(-lo / s), 0, Q),  q = clamp(rint(w / s) + z, 0, Q)
+ *   ternary: a = (|w_0| + |w_1| + ... + |w_127|) / 128, summed left to right
+ *            s = fp16_rne(a), s := 1 if s == 0,  t = clamp(rint(w / s), -1, 1)
+ * fp16_rne is the direct float64 -> binary16 rounding (never through float32).
+ * Inputs must be finite.
+ *
+ * Layouts (all row-major, rows contiguous; G = K / 128):
+ *   int4 codes   uint32 [N, K/8]    code k in word k/8,  bits 4*(k%8)..4*(k%8)+3
+ *   int2 codes   uint32 [N, K/16]   code k in word k/16, bits 2*(k%16)..2*(k%16)+1
+ *   ternary      uint8  [N, 26*G]   group g of a row at bytes 26g..26g+25; byte j of a
+ *                                   group = sum_{i<5} (t_{5j+i} + 1) * 3^i; byte 25 holds
+ *                                   trits 125..127 and two pad trits 0 (digit 1); every
+ *                                   byte is in 0..242
+ *   scale, zero  fp16 bits (uint16) [N, G]; zero is unused (NULL) for WQ_TERNARY
+ *   x, X, y, Y   fp16 bits (uint16), X [M, K] and Y [M, N] row-major
+ *
+ * Conventions.
+ *   - Every pointer argument except `stream` is a DEVICE pointer owned by the caller;
+ *     the library allocates no device memory and keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Work is enqueued asynchronously; a call returns once its kernels are launched.
+ *   - Errors are returned as wq_status, never thrown. All argument checks happen before
+ *     any launch: on a non-WQ_OK return from a check, nothing was enqueued and no
+ *     output was touched. WQ_ERR_CUDA means a launch failed; outputs are then undefined.
+ *   - Requirements: 1 <= N <= 2^31 - 1, 128 <= K <= 2^20 - 128 and K % 128 == 0;
+ *     W (for wq_quantize), codes, x/X and y/Y 16-byte aligned; scale and zero 2-byte
+ *     aligned; buffers may not overlap except inputs shared between calls.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { WQ_INT4 = 0, WQ_INT2 = 1, WQ_TERNARY = 2 } wq_fmt;
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_ARG = 1,          /* null pointer, unknown format, group != 128 */
+  WQ_ERR_SHAPE = 2,        /* N, K or M outside the supported range, K % 128 != 0 */
+  WQ_ERR_ALIGN = 3,        /* a pointer is not aligned as required above */
+  WQ_ERR_CUDA = 4,         /* a CUDA call or launch failed (see wq_last_cuda_error) */
+  WQ_ERR_UNSUPPORTED = 5   /* valid request this build cannot serve (e.g. no sm_100 GPU) */
+} wq_status;
+
+/* Bytes of packed codes for an [N, K] weight in format fmt (0 on invalid arguments):
+ * int4 N*K/2, int2 N*K/4, ternary N*26*(K/128). */
+size_t wq_codes_bytes(int fmt, int64_t N, int64_t K);
+
+/* Number of fp16 entries of the scale array (and of the zero array): N * K / 128. */
+size_t wq_meta_count(int64_t N, int64_t K);
+
+/* Quantise W (fp32 [N, K], device) into codes / scale / zero as defined above.
+ * group must be 128. zero must be NULL for WQ_TERNARY and non-NULL otherwise.
+ * Whetstone README, "What the weights can actually survive" (round-to-nearest group
+ * quantisation) and TKintegers K5, "What is K5?" (base-3 trit bytes). */
+int wq_quantize(const float* W, int64_t N, int64_t K, int fmt, int group,
+                void* codes, uint16_t* scale, uint16_t* zero, void* stream);
+
+/* y[n] = fp16( sum_k x[k] * w_hat[n, k] ), fp32 accumulation, for one activation vector
+ * x (fp16 [K]); y is fp16 [N]. Whetstone README, "The one fact that shapes everything"
+ * (each weight read once, one multiply-add per weight). */
+int wq_gemv(const uint16_t* x, const void* codes, const uint16_t* scale,
+            const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* y,
+            void* stream);
+
+/* Y[m, n] = fp16( sum_k X[m, k] * w_hat[n, k] ) for M activation rows, 1 <= M <= 2048.
+ * M = 1 runs the wq_gemv kernel. Small M streams the weights once and reuses each
+ * dequantised weight for every row of X; large M dequantises weight tiles into shared
+ * memory as fp16 tensor-core operands with fp32 accumulators (TKintegers K5, "What is
+ * K5?": tiles expanded to fp16 tensor-core operands, fp32 accumulation). */
+int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* scale,
+            const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* Y,
+            void* stream);
+
+/* One matrix of a linear set: y = x . w_hat^T with this matrix's own x and y. */
+typedef struct {
+  const void* codes;
+  const uint16_t* scale;
+  const uint16_t* zero;   /* NULL for WQ_TERNARY */
+  const uint16_t* x;      /* fp16 [K] */
+  uint16_t* y;            /* fp16 [N] */
+  int64_t N;
+  int64_t K;
+} wq_linear_desc;
+
+/* Largest count accepted by wq_linear_set. */
+#define WQ_LINEAR_SET_MAX 256
+
+/* Run `count` independent matrix-vector products of one format in ONE persistent kernel
+ * launch. `descs` is a HOST array (read during the call, not kept); the pointers inside
+ * are device pointers. Equivalent to count wq_gemv calls, without count launches: at
+ * batch 1 a whole decoded token reads every weight once, and per-launch overhead
+ * dominates small matrices (Whetstone README, "The baseline, and where the opportunity
+ * actually is": dispatch and launch overhead, not bytes, set the baseline's speed).
+ * 1 <= count <= WQ_LINEAR_SET_MAX; each entry obeys the wq_gemv requirements. */
+int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream);
+
+/* Static string naming a status code. */
+const char* wq_status_str(int status);
+
+/* The cudaError_t value of the last WQ_ERR_CUDA in this thread (0 if none). */
+int wq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

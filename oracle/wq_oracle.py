@@ -4,9 +4,10 @@ TEST INFRASTRUCTURE ONLY. Nothing in the product path may import, call or execut
 module: only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline / reference leg
 use it. It shares no code with the CUDA path.
 
-It follows the Whetstone README ("Evaluation harness": a deliberately slow and obvious
-float64 reference that is trusted over the fast kernel; "Quality gates" item 1: kernel
-output must match a CPU reference within a stated tolerance). Everything is numpy in
+It follows the Whetstone README: its "Evaluation harness" section keeps a float64
+reference with no fusion or shortcuts, and trusts it over any fast kernel that disagrees;
+its "Quality gates" section requires kernel output to agree with a CPU reference within
+a stated tolerance. Everything is numpy in
 float64. Where the pages leave a step open, the plainest reading is taken and marked
 READING in the function's docstring.
 
@@ -77,16 +78,16 @@ def f16_from_bits(b) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
-# Quantisers.  Whetstone README, "What the weights can actually survive": round-to-nearest,
-# group 128, "an f16 scale plus an f16 zero" per group (0.25 bits/weight of metadata);
-# format table rows int4 g128 (4.25), int2 g128 (2.25), ternary g128 (1.71).
+# Quantisers.  Whetstone README, "What the weights can actually survive": round-to-nearest
+# at group 128, with one fp16 scale and one fp16 zero per group (0.25 bits/weight of
+# metadata); format table rows int4 g128 (4.25), int2 g128 (2.25), ternary g128 (1.71).
 # --------------------------------------------------------------------------------------
 
 def quantize_int(W, bits: int):
     """Asymmetric round-to-nearest group-128 quantisation along K to `bits`-bit codes.
 
-    READING (the pages name RTN, asymmetric, group 128 and an fp16 scale + fp16 zero but
-    give no formula); per (row n, group g), with Q = 2^bits - 1 and w in float64:
+    READING (the pages name round-to-nearest, asymmetric, group 128 and fp16 scale and
+    zero, but give no formula); per (row n, group g), with Q = 2^bits - 1 and w in float64:
         lo = min w, hi = max w
         s  = fp16(( hi - lo) / Q);  s = 1 if that is 0 (constant group / underflow)
         z  = clamp(rint(-lo / s), 0, Q)          (integer zero point, stored as fp16)
@@ -105,7 +106,7 @@ def quantize_int(W, bits: int):
     hi = w.max(axis=2)
     s = f16_round((hi - lo) / Q)
     s = np.where(s == 0.0, 1.0, s)
-    z = np.clip(np.rint(-lo / s), 0.0, Q)
+    z = np.clip(np.rint(-lo / s), 0.0, Q) + 0.0          # an integer: no negative zero
     q = np.clip(np.rint(w / s[:, :, None]) + z[:, :, None], 0.0, Q).astype(np.uint32)
     return pack_int(q.reshape(N, K), bits), f16_to_bits(s), f16_to_bits(z)
 
@@ -142,8 +143,8 @@ def dequant_int(codes, scale_bits, zero_bits, bits: int, K: int) -> np.ndarray:
     return (q - z) * s
 
 
-# Ternary.  TKintegers K5, "What is K5?": five balanced-ternary digits per one-byte code,
-# 243 values ("five trits does not mean five binary bits").  READING: the byte holds five
+# Ternary.  TKintegers K5, "What is K5?": a one-byte code made of five balanced-ternary
+# digits, so 243 values (trits, not bits).  READING: the byte holds five
 # ternary WEIGHTS t_0..t_4 in {-1, 0, +1} as the base-3 number sum_i (t_i + 1) 3^i, lowest
 # weight in the least significant digit.
 TRITS_PER_BYTE = 5

@@ -1,0 +1,87 @@
+"""The C-ABI library loads and exports every entry point wq.h declares (no GPU needed).
+
+Only host-side logic is exercised: size queries and the argument checks that reject a
+call before anything touches CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_weight_quantized_unpack_b200 import build as wq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ctypes.CDLL(wq_build.build())
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(wq_\w+)\s*\(", src, re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"wq_quantize", "wq_gemv", "wq_gemm", "wq_linear_set", "wq_codes_bytes",
+            "wq_meta_count", "wq_status_str", "wq_last_cuda_error"} <= names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_sizes(lib):
+    lib.wq_codes_bytes.restype = ctypes.c_size_t
+    lib.wq_codes_bytes.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64]
+    lib.wq_meta_count.restype = ctypes.c_size_t
+    lib.wq_meta_count.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    assert lib.wq_codes_bytes(0, 151936, 896) == 151936 * 448
+    assert lib.wq_codes_bytes(1, 151936, 896) == 151936 * 224
+    assert lib.wq_codes_bytes(2, 151936, 896) == 151936 * 182
+    assert lib.wq_meta_count(151936, 896) == 151936 * 7
+    # stored bits per weight of the layout: 4.25, 2.25, 1.75
+    for fmt, bpw in ((0, 4.25), (1, 2.25), (2, 1.75)):
+        meta_arrays = 1 if fmt == 2 else 2          # scale (+ zero), fp16 each
+        tot = lib.wq_codes_bytes(fmt, 64, 1024) + 2 * meta_arrays * lib.wq_meta_count(64, 1024)
+        assert tot * 8 / (64 * 1024) == bpw
+    assert lib.wq_codes_bytes(0, 4, 100) == 0      # K not a multiple of 128
+    assert lib.wq_codes_bytes(3, 4, 128) == 0      # unknown format
+    assert lib.wq_codes_bytes(0, 0, 128) == 0
+
+
+def test_argument_checks_reject_before_any_launch(lib):
+    from bit_weight_quantized_unpack_b200 import wq
+    P = 1 << 20   # a 16-byte aligned fake address: never dereferenced on a rejected call
+    S = None      # stream
+    # null pointers, bad format, bad group
+    assert wq._lib.wq_gemv(None, P, P, P, 0, 8, 128, P, S) == wq.WQ_ERR_ARG
+    assert wq._lib.wq_gemv(P, P, P, None, 0, 8, 128, P, S) == wq.WQ_ERR_ARG      # int4 needs zero
+    assert wq._lib.wq_gemv(P, P, P, P, 2, 8, 128, P, S) == wq.WQ_ERR_ARG         # ternary: no zero
+    assert wq._lib.wq_gemv(P, P, P, P, 7, 8, 128, P, S) == wq.WQ_ERR_ARG
+    assert wq._lib.wq_quantize(P, 8, 128, 0, 64, P, P, P, S) == wq.WQ_ERR_ARG
+    # shapes
+    assert wq._lib.wq_gemv(P, P, P, P, 0, 8, 100, P, S) == wq.WQ_ERR_SHAPE
+    assert wq._lib.wq_gemv(P, P, P, P, 0, 0, 128, P, S) == wq.WQ_ERR_SHAPE
+    assert wq._lib.wq_gemv(P, P, P, P, 0, 8, 0, P, S) == wq.WQ_ERR_SHAPE
+    assert wq._lib.wq_gemm(P, 0, P, P, P, 0, 8, 128, P, S) == wq.WQ_ERR_SHAPE
+    assert wq._lib.wq_gemm(P, 2049, P, P, P, 0, 8, 128, P, S) == wq.WQ_ERR_SHAPE
+    # alignment
+    assert wq._lib.wq_gemv(P + 8, P, P, P, 0, 8, 128, P, S) == wq.WQ_ERR_ALIGN
+    assert wq._lib.wq_gemv(P, P + 4, P, P, 0, 8, 128, P, S) == wq.WQ_ERR_ALIGN
+    assert wq._lib.wq_gemv(P, P, P + 1, P, 0, 8, 128, P, S) == wq.WQ_ERR_ALIGN
+    assert wq._lib.wq_quantize(P + 4, 8, 128, 0, 128, P, P, P, S) == wq.WQ_ERR_ALIGN
+    # linear set: count range, and a bad entry anywhere rejects the whole call
+    good = (P, P, P, P, P, 8, 128)
+    arr = wq.make_linear_set([good, (P, P, P, P, P, 8, 130)])
+    assert wq._lib.wq_linear_set(arr, 2, 0, S) == wq.WQ_ERR_SHAPE
+    assert wq._lib.wq_linear_set(arr, 0, 0, S) == wq.WQ_ERR_ARG
+    assert wq._lib.wq_linear_set(arr, 257, 0, S) == wq.WQ_ERR_ARG
+    assert wq._lib.wq_linear_set(None, 1, 0, S) == wq.WQ_ERR_ARG
+    assert wq.wq_status_str(wq.WQ_ERR_ALIGN).startswith("WQ_ERR_ALIGN")
