@@ -1,0 +1,37 @@
+// Parameters of the tensor-core dequantising GEMM (gemm_tc.cu) and its host entry points.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wq {
+
+constexpr int kTcMaxBN = 256;   // tokens per tile (MMA N), also the TMEM columns allocated
+constexpr int kTcMaxMats = 64;  // matrices per launch (tensor maps travel as kernel params)
+constexpr int kTcMinM = 16;     // wq_gemm uses the tensor-core path from this M up (int4)
+
+// One matrix: tiles [tile_begin, tile_end) of the launch, tiles_m token tiles per
+// 128-row weight tile. Tensor maps first: CUtensorMap needs 64-byte alignment.
+struct TcMat {
+  CUtensorMap tmap_x;      // X [M, K] fp16, box 64 x bn, 128-byte swizzle
+  CUtensorMap tmap_codes;  // int4 codes as bytes [N, K/2], box 32 x 128
+  const uint16_t* scale;
+  const uint16_t* zero;
+  uint16_t* y;             // fp16 [M, ldy]
+  int N, K, M, ldy, bn, tiles_n, tiles_m, tile_begin, tile_end;
+};
+
+struct TcParams {
+  TcMat m[kTcMaxMats];
+  int count;
+  int total_tiles;
+};
+
+bool tc_plan_mat(TcMat& t, const uint16_t* X, int M, const void* codes, const uint16_t* scale,
+                 const uint16_t* zero, uint16_t* Y, int N, int K, int bn);
+int tc_bn_for(int M);
+cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream);
+cudaError_t read_device_errors(unsigned int* flags, bool clear, cudaStream_t stream);
+
+}  // namespace wq

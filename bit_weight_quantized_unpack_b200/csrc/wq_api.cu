@@ -3,6 +3,7 @@
 #include <limits.h>
 #include <string.h>
 
+#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "wq.h"
 
@@ -106,6 +107,18 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
   if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
   if (!aligned(X, 16) || !aligned(Y, 2)) return WQ_ERR_ALIGN;
   if ((st = check_device()) != WQ_OK) return st;
+  if (fmt == WQ_INT4 && M >= wq::kTcMinM) {
+    // tensor-core path: 128-row weight tiles x up to 256 tokens
+    static thread_local wq::TcParams tp;  // ~20 KB: kept off the stack, one per thread
+    const int bn = wq::tc_bn_for((int)M);
+    if (!wq::tc_plan_mat(tp.m[0], X, (int)M, codes, scale, zero, Y, (int)N, (int)K, bn))
+      return WQ_ERR_CUDA;
+    tp.m[0].tile_begin = 0;
+    tp.m[0].tile_end = tp.m[0].tiles_n * tp.m[0].tiles_m;
+    tp.count = 1;
+    tp.total_tiles = tp.m[0].tile_end;
+    return cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
+  }
   wq::SetParams p;
   p.count = 1;
   const int64_t items = plan_mat(p.m[0], fmt, codes, scale, zero, X, Y, N, K, M);
@@ -163,5 +176,12 @@ const char* wq_status_str(int status) {
 }
 
 int wq_last_cuda_error(void) { return g_last_cuda_error; }
+
+int wq_device_errors(unsigned int* flags, int clear, void* stream) {
+  if (!flags) return WQ_ERR_ARG;
+  int st = check_device();
+  if (st != WQ_OK) return st;
+  return cuda_status(wq::read_device_errors(flags, clear != 0, (cudaStream_t)stream));
+}
 
 }  // extern "C"

@@ -42,6 +42,7 @@ _sig = {
     "wq_linear_set": (_i, [ctypes.POINTER(wq_linear_desc), _i, _i, _p]),
     "wq_status_str": (ctypes.c_char_p, [_i]),
     "wq_last_cuda_error": (_i, []),
+    "wq_device_errors": (_i, [ctypes.POINTER(ctypes.c_uint), _i, _p]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -123,6 +124,16 @@ def wq_status_str(status: int) -> str:
 
 def wq_last_cuda_error() -> int:
     return _lib.wq_last_cuda_error()
+
+
+def wq_device_errors(clear: bool = True, stream=None) -> int:
+    """Device error flags (WQ_DEVERR_*) since the last clear; synchronises the stream."""
+    f = ctypes.c_uint(0)
+    _check(_lib.wq_device_errors(ctypes.byref(f), int(clear), _stream(stream)), "wq_device_errors")
+    return f.value
+
+
+WQ_DEVERR_TIMEOUT = 1
 
 
 # ---- allocation helpers (torch owns the memory) ------------------------------------

@@ -129,6 +129,13 @@ const char* wq_status_str(int status);
 /* The cudaError_t value of the last WQ_ERR_CUDA in this thread (0 if none). */
 int wq_last_cuda_error(void);
 
+/* Device-side error flags of this library on the current device, OR-ed over every kernel
+ * since the last clear: bit 0 (WQ_DEVERR_TIMEOUT) = a bounded wait inside a tensor-core
+ * kernel gave up (its outputs are then undefined; the kernel freed its resources and
+ * returned instead of hanging). Synchronises `stream`; clears the flags if clear != 0. */
+#define WQ_DEVERR_TIMEOUT 1u
+int wq_device_errors(unsigned int* flags, int clear, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
