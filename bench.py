@@ -222,7 +222,47 @@ def bench_rows(args, pk):
                                        "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"]}
         del copies
         torch.cuda.empty_cache()
+    rows.update(bench_batch_sweep(args, pk))
     return rows
+
+
+def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 64, 512, 2048)):
+    """Batch sweep on the 0.5B set: one wq_gemm per matrix, the 169 calls in a CUDA graph."""
+    from bit_weight_quantized_unpack_b200 import wq
+    wl = workloads.WORKLOADS[4]
+    mats = workloads.workload_mats(4)
+    packed = []
+    for i, m in enumerate(mats):
+        W = synth.weights(m.N, m.K, wl["sigma"], synth.sub_seed(wl["seed"], i, 0), device="cuda")
+        c, s, z = wq.alloc_packed(m.N, m.K, "int4")
+        wq.wq_quantize(W, m.N, m.K, "int4", 128, c, s, z)
+        del W
+        packed.append((c, s, z))
+    weights = sum(m.N * m.K for m in mats)
+    out = {}
+    for M in Ms:
+        X = [synth.activations(M, m.K, synth.sub_seed(wl["seed"], i, 1), device="cuda")
+             for i, m in enumerate(mats)]
+        Y = [torch.empty(M, m.N, dtype=torch.float16, device="cuda") for m in mats]
+
+        def one_pass():
+            for (c, s, z), m, x, y in zip(packed, mats, X, Y):
+                wq.wq_gemm(x, M, c, s, z, "int4", m.N, m.K, y)
+        one_pass()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one_pass()
+        steps = 20 if M >= 512 else 50
+        ms = time_steps(lambda i: g.replay(), steps if not args.quick else 5, 3, 1)
+        flops = 2.0 * M * weights
+        out[f"gemm_set_M{M}"] = {"ms": ms, "TFLOPS": flops / ms / 1e9,
+                                 "frac_tensor": flops / ms / 1e9 / pk["bf16_tflops"],
+                                 "weight_GBps": weights * INT4_BYTES_PER_WEIGHT / ms / 1e6,
+                                 "launches_per_pass": len(mats)}
+        del g, X, Y
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -275,13 +315,18 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(nbytes / ms / 1e6, 2),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(nbytes / ms / 1e6 / pk["hbm_gbs"], 4),
-                         "traffic": None, "kernel": "gemv_int_set_kernel<4,1>",
+                         "traffic": None, "kernel": "gemv_bulk_kernel<4>",
                          "peak_source": pk["source"]},
             "e2e": {"value": round(nbytes * ws / ms_e2e / 1e6, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * K_tot, "d2h_bytes_per_step": 2 * N_tot},
             "gpu_launches": args.steps,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
+            "gemm_m512": ({"TFLOPS": round(rows["gemm_set_M512"]["TFLOPS"], 1),
+                           "frac_of_tensor_peak": round(rows["gemm_set_M512"]["frac_tensor"], 4),
+                           "peak_tflops": pk["bf16_tflops"],
+                           "workload": "qwen2.5-0.5b set, M=512, one wq_gemm per matrix in a CUDA graph"}
+                          if "gemm_set_M512" in rows else None),
             "rows": rows,
         }
         print(json.dumps(line), flush=True)

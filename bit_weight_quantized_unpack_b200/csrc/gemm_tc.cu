@@ -313,6 +313,18 @@ cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+unsigned int* device_error_word() {
+  static unsigned int* addr[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_errors) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return addr[dev];
+}
+
 cudaError_t read_device_errors(unsigned int* flags, bool clear, cudaStream_t stream) {
   cudaError_t e = cudaMemcpyFromSymbolAsync(flags, g_device_errors, sizeof(unsigned int), 0,
                                             cudaMemcpyDeviceToHost, stream);

@@ -33,5 +33,7 @@ bool tc_plan_mat(TcMat& t, const uint16_t* X, int M, const void* codes, const ui
 int tc_bn_for(int M);
 cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream);
 cudaError_t read_device_errors(unsigned int* flags, bool clear, cudaStream_t stream);
+// Device address of the error word on the current device (looked up once per device).
+unsigned int* device_error_word();
 
 }  // namespace wq

@@ -5,6 +5,7 @@
 
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_bulk.cuh"
 #include "wq.h"
 
 namespace {
@@ -71,6 +72,32 @@ int64_t plan_mat(wq::SetMat& m, int fmt, const void* codes, const uint16_t* scal
   return (N + rows - 1) / rows;
 }
 
+// Plan the bulk-staged kernel for entries [0, count) of a set (int4 / int2, batch 1).
+// Returns false if any matrix needs the register-streaming kernel instead.
+bool plan_bulk(wq::BulkParams& p, int fmt, int count, const wq_linear_desc* d) {
+  if (fmt == WQ_TERNARY || count > wq::kBulkMaxMats) return false;
+  const int bits = fmt == WQ_INT4 ? 4 : 2;
+  p.errors = wq::device_error_word();
+  if (!p.errors) return false;
+  p.count = count;
+  int64_t blocks = 0, cost = 0;
+  for (int i = 0; i < count; ++i) {
+    wq::BulkMat& m = p.m[i];
+    if (!wq::bulk_plan_mat(m, bits, d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K))
+      return false;
+    const int64_t nb = (d[i].N + m.rows_per_block - 1) / m.rows_per_block;
+    m.block_begin = (int)blocks;
+    m.cost_begin = cost;
+    blocks += nb;
+    cost += nb * m.block_bytes;
+    if (blocks > INT_MAX) return false;
+    m.block_end = (int)blocks;
+  }
+  p.total_blocks = (int)blocks;
+  p.total_cost = cost;
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -119,6 +146,11 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
     tp.total_tiles = tp.m[0].tile_end;
     return cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
   }
+  if (M == 1 && fmt != WQ_TERNARY) {
+    static thread_local wq::BulkParams bp;
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K};
+    if (plan_bulk(bp, fmt, 1, &d)) return cuda_status(wq::launch_gemv_bulk(bp, fmt == WQ_INT4 ? 4 : 2, (cudaStream_t)stream));
+  }
   wq::SetParams p;
   p.count = 1;
   const int64_t items = plan_mat(p.m[0], fmt, codes, scale, zero, X, Y, N, K, M);
@@ -152,6 +184,13 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
     total += items;
     if (total > INT_MAX) return WQ_ERR_SHAPE;
     p.m[i].item_end = (int)total;
+  }
+  int st0 = check_device();
+  if (st0 != WQ_OK) return st0;
+  {
+    static thread_local wq::BulkParams bp;
+    if (plan_bulk(bp, fmt, count, descs))
+      return cuda_status(wq::launch_gemv_bulk(bp, fmt == WQ_INT4 ? 4 : 2, (cudaStream_t)stream));
   }
   for (int i = count; i < wq::kSetMax; ++i) {
     memset(&p.m[i], 0, sizeof(p.m[i]));
