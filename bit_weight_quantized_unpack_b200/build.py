@@ -45,7 +45,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         o = os.path.join(BUILD, src[:-3] + ".o")
         objs.append(o)
         if force or _stale(o, [s, __file__] + hdrs):
-            cmd = [NVCC] + COMMON + EXTRA.get(src, []) + ["-c", s, "-o", o]
+            cmd = [NVCC] + COMMON + EXTRA.get(src, []) + os.environ.get("WQ_NVCC_EXTRA", "").split() + ["-c", s, "-o", o]
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
                 print(" ".join(cmd), flush=True)

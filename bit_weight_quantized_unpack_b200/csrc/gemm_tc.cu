@@ -36,19 +36,22 @@ namespace {
 
 constexpr int BM = 128;       // weight rows per tile
 constexpr int BK = 64;        // k per stage: one 128-byte swizzle row of fp16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;            // 16 KB
-constexpr int B_BYTES = kTcMaxBN * BK * 2;      // 32 KB
+constexpr int TSTAGES = 5;    // TMA ring: activation tile + codes of one k-block
+constexpr int ASTAGES = 2;    // dequantised weight tiles (written by CUDA cores, read by MMA)
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB of dequantised fp16 weights
+constexpr int B_BYTES = kTcMaxBN * BK * 2;      // 32 KB of activations
 constexpr int C_BYTES = BM * BK / 2;            // 4 KB of int4 codes
+constexpr int T_BYTES = B_BYTES + C_BYTES;      // one TMA stage
 constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_BAR = OFF_C + STAGES * C_BYTES;
-constexpr int NUM_BARS = 3 * STAGES + 1;
+constexpr int OFF_T = OFF_A + ASTAGES * A_BYTES;
+constexpr int OFF_BAR = OFF_T + TSTAGES * T_BYTES;
+constexpr int NUM_BARS = 2 * TSTAGES + 2 * ASTAGES + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
-constexpr int DEQ_THREADS = 256;
-constexpr int THREADS = 384;
+constexpr int THREADS = 512;                    // 16 warps
+constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, DEQ_WARP0 = 8, DEQ_WARPS = 8;
+constexpr int TMEM_COLS = 2 * kTcMaxBN;         // two accumulator buffers
+static_assert(T_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzled operands need 1 KB alignment");
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
@@ -78,46 +81,77 @@ __device__ __forceinline__ uint4 dequant8(uint32_t v, uint32_t c1024z, uint32_t 
   return r;
 }
 
+// First tile whose starting cost is >= target (tiles of all matrices numbered in order).
+__device__ int first_tile_at(const TcParams& P, int64_t target) {
+  for (int i = 0; i < P.count; ++i) {
+    const TcMat& m = P.m[i];
+    const int64_t end = m.cost_begin + (int64_t)(m.tile_end - m.tile_begin) * m.tile_cost;
+    if (target < end) {
+      const int64_t off = target - m.cost_begin;
+      const int64_t j = off <= 0 ? 0 : (off + m.tile_cost - 1) / m.tile_cost;
+      return m.tile_begin + (int)j;
+    }
+  }
+  return P.total_tiles;
+}
+
+struct TileInfo {
+  int mi, n0, m0, bn, nkb;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const TcParams& P, int tile, int& mi) {
+  while (tile >= P.m[mi].tile_end) ++mi;
+  const TcMat& M = P.m[mi];
+  const int local = tile - M.tile_begin;
+  TileInfo t;
+  t.mi = mi;
+  t.n0 = (local / M.tiles_m) * BM;
+  t.m0 = (local % M.tiles_m) * M.bn;
+  t.bn = M.bn;
+  t.nkb = M.K / BK;
+  return t;
+}
+
 }  // namespace
 
+// Persistent: CTA b runs the tiles whose starting cost lies in its 1/gridDim share, in
+// order. Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31 = weight rows), 4 TMA producer,
+// 5 MMA issuer (and TMEM owner), 8-15 dequantisers (two threads per weight row, 32 k each
+// per stage); 6-7 idle. The two 256-column TMEM accumulators let the epilogue of one tile
+// overlap the main loop of the next.
 __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_constant__ TcParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment of the operand buffers is what the 128-byte swizzle assumes
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = tc::smem_u32(smem);
-  const uint32_t bar_full = sbase + OFF_BAR;                 // [STAGES]
-  const uint32_t bar_aready = bar_full + 8 * STAGES;         // [STAGES]
-  const uint32_t bar_empty = bar_aready + 8 * STAGES;        // [STAGES]
-  const uint32_t bar_tmem = bar_empty + 8 * STAGES;          // [1]
+  const uint32_t bar_full = sbase + OFF_BAR;                  // [TSTAGES] TMA: X tile + codes landed
+  const uint32_t bar_empty = bar_full + 8 * TSTAGES;          // [TSTAGES] MMAs reading it done
+  const uint32_t bar_aready = bar_empty + 8 * TSTAGES;        // [ASTAGES] dequantised A written
+  const uint32_t bar_aempty = bar_aready + 8 * ASTAGES;       // [ASTAGES] MMAs reading A done
+  const uint32_t bar_tfull = bar_aempty + 8 * ASTAGES;        // [2] accumulator complete
+  const uint32_t bar_tempty = bar_tfull + 16;                 // [2] accumulator drained
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);  // [0] tmem base, [1] abort
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- which tile ----
-  const int tile = blockIdx.x;
-  int mi = 0;
-  while (tile >= P.m[mi].tile_end) ++mi;
-  const TcMat& M = P.m[mi];
-  const int local = tile - M.tile_begin;
-  const int n0 = (local / M.tiles_m) * BM;
-  const int m0 = (local % M.tiles_m) * M.bn;
-  const int BN = M.bn;
-  const int nkb = M.K / BK;
-
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < TSTAGES; ++i) {
       tc::mbar_init(bar_full + 8 * i, 1);
-      tc::mbar_init(bar_aready + 8 * i, DEQ_THREADS / 32);
       tc::mbar_init(bar_empty + 8 * i, 1);
     }
-    tc::mbar_init(bar_tmem, 1);
+    for (int i = 0; i < ASTAGES; ++i) {
+      tc::mbar_init(bar_aready + 8 * i, DEQ_WARPS);
+      tc::mbar_init(bar_aempty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(bar_tfull + 8 * i, 1);
+      tc::mbar_init(bar_tempty + 8 * i, 4);
+    }
     tc::fence_mbar_init();
     misc[1] = 0;
-    tc::prefetch_tmap(&M.tmap_x);
-    tc::prefetch_tmap(&M.tmap_codes);
   }
-  if (warp == 1) {
-    tc::tmem_alloc(sbase + OFF_MISC, kTcMaxBN);  // 256 fp32 columns x 128 lanes
+  if (warp == MMA_WARP) {
+    tc::tmem_alloc(sbase + OFF_MISC, TMEM_COLS);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -125,98 +159,150 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   tc::tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  bool timed_out = false;
-  int issued = 0;  // TMA stages issued by the producer (drained on the error path)
+  const int64_t share = (P.total_cost + gridDim.x - 1) / gridDim.x;
+  const int t_lo = first_tile_at(P, share * blockIdx.x);
+  const int t_hi = first_tile_at(P, share * (blockIdx.x + 1));
 
-  if (warp == 0) {
-    // ---------------- producer ----------------
+  bool timed_out = false;
+  int it = 0;  // k-block sequence number over this CTA's tiles
+  int mi = 0;
+
+  if (warp == PRODUCER_WARP) {
     if (lane == 0) {
-      const uint32_t tx = (uint32_t)(BN * BK * 2 + C_BYTES);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!tc::mbar_wait(bar_empty + 8 * s, ph ^ 1)) { timed_out = true; break; }
-        if (misc[1]) break;
-        tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
-        tc::tma_load_2d(sbase + OFF_B + s * B_BYTES, &M.tmap_x, bar_full + 8 * s, kb * BK, m0);
-        tc::tma_load_2d(sbase + OFF_C + s * C_BYTES, &M.tmap_codes, bar_full + 8 * s, kb * (BK / 2), n0);
-        ++issued;
+      for (int tile = t_lo; tile < t_hi && !timed_out; ++tile) {
+        const TileInfo ti = tile_info(P, tile, mi);
+        const TcMat& M = P.m[ti.mi];
+        const uint32_t tx = (uint32_t)(ti.bn * BK * 2 + C_BYTES);
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+          const int s = it % TSTAGES;
+          if (!tc::mbar_wait(bar_empty + 8 * s, ((it / TSTAGES) & 1) ^ 1)) { timed_out = true; break; }
+          if (misc[1]) { timed_out = true; break; }
+          const uint32_t st = sbase + OFF_T + s * T_BYTES;
+          tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+          tc::tma_load_2d(st, &M.tmap_x, bar_full + 8 * s, kb * BK, ti.m0);
+          tc::tma_load_2d(st + B_BYTES, &M.tmap_codes, bar_full + 8 * s, kb * (BK / 2), ti.n0);
+        }
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == MMA_WARP) {
     if (lane == 0) {
-      const uint32_t idesc = tc::idesc_f16_f32(BM, BN);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!tc::mbar_wait(bar_full + 8 * s, ph) || !tc::mbar_wait(bar_aready + 8 * s, ph)) {
+      int lt = 0;
+      for (int tile = t_lo; tile < t_hi && !timed_out; ++tile, ++lt) {
+        const TileInfo ti = tile_info(P, tile, mi);
+        const int b = lt & 1;
+        if (!tc::mbar_wait(bar_tempty + 8 * b, ((lt >> 1) & 1) ^ 1)) { timed_out = true; break; }
+        tc::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(b * kTcMaxBN);
+        const uint32_t idesc = tc::idesc_f16_f32(BM, ti.bn);
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+          const int s = it % TSTAGES, a = it % ASTAGES;
+          if (!tc::mbar_wait(bar_full + 8 * s, (it / TSTAGES) & 1) ||
+              !tc::mbar_wait(bar_aready + 8 * a, (it / ASTAGES) & 1)) {
+            timed_out = true;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint64_t ad = tc::sw128_kmajor_desc(sbase + OFF_A + a * A_BYTES);
+          const uint64_t bd = tc::sw128_kmajor_desc(sbase + OFF_T + s * T_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)  // +32 bytes along K inside the swizzled row
+            tc::mma_f16_ss(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+          tc::mma_commit(bar_empty + 8 * s);   // frees the TMA stage ...
+          tc::mma_commit(bar_aempty + 8 * a);  // ... and the dequantised tile
+        }
+        tc::mma_commit(bar_tfull + 8 * b);  // fires when every MMA of the tile has completed
+      }
+    }
+  } else if (warp >= DEQ_WARP0) {
+    // two threads per weight row: thread pairs (2r, 2r+1) take k 0..31 and 32..63 of it
+    const int t = threadIdx.x - 32 * DEQ_WARP0;
+    const int r = t >> 1, h = t & 1;
+    // scale | zero << 16 of groups g, g+1 (loaded ahead); the next tile's first two groups
+    // are fetched near the end of the current tile so a tile start never waits on them
+    auto load_sz = [&](const TcMat& M, int n, int g) -> uint32_t {
+      const int G = M.K / kGroup;
+      return (uint32_t)ld_u16(M.scale + (size_t)n * G + g) | ((uint32_t)ld_u16(M.zero + (size_t)n * G + g) << 16);
+    };
+    uint32_t pre0 = 0, pre1 = 0;
+    int mi_pre = 0;
+    if (t_lo < t_hi) {
+      const TileInfo t0 = tile_info(P, t_lo, mi_pre);
+      const TcMat& M0 = P.m[t0.mi];
+      const int n = min(t0.n0 + r, M0.N - 1);
+      pre0 = load_sz(M0, n, 0);
+      pre1 = M0.K > kGroup ? load_sz(M0, n, 1) : 0u;
+    }
+    for (int tile = t_lo; tile < t_hi && !timed_out; ++tile) {
+      const TileInfo ti = tile_info(P, tile, mi);
+      const TcMat& M = P.m[ti.mi];
+      const int n = min(ti.n0 + r, M.N - 1);  // rows past N are computed but never stored
+      const int G = M.K / kGroup;
+      uint32_t sz0 = pre0, sz1 = pre1, sz2 = 0;
+      uint32_t c1024z = 0, s2 = 0;
+      const int kb_pre = ti.nkb > 4 ? ti.nkb - 4 : 0;
+      for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+        const int s = it % TSTAGES, a = it % ASTAGES;
+        if ((kb & 1) == 0) {
+          const int g = kb >> 1;
+          if (g + 2 < G) sz2 = load_sz(M, n, g + 2);
+          const __half z = __ushort_as_half((uint16_t)(sz0 >> 16));
+          c1024z = pack_h2(__hadd(z, __float2half(1024.f)));
+          s2 = (sz0 & 0xFFFFu) | (sz0 << 16);
+          sz0 = sz1;
+          sz1 = sz2;
+        }
+        if (kb == kb_pre && tile + 1 < t_hi) {
+          const TileInfo tn = tile_info(P, tile + 1, mi_pre);
+          const TcMat& Mn = P.m[tn.mi];
+          const int nn = min(tn.n0 + r, Mn.N - 1);
+          pre0 = load_sz(Mn, nn, 0);
+          pre1 = Mn.K > kGroup ? load_sz(Mn, nn, 1) : 0u;
+        }
+        if (!tc::mbar_wait(bar_full + 8 * s, (it / TSTAGES) & 1) ||
+            !tc::mbar_wait(bar_aempty + 8 * a, ((it / ASTAGES) & 1) ^ 1)) {
           timed_out = true;
           break;
         }
-        tc::tc_fence_after();
-        const uint64_t ad = tc::sw128_kmajor_desc(sbase + OFF_A + s * A_BYTES);
-        const uint64_t bd = tc::sw128_kmajor_desc(sbase + OFF_B + s * B_BYTES);
+        const uint4 cw = *reinterpret_cast<const uint4*>(smem + OFF_T + s * T_BYTES + B_BYTES + r * 32 + h * 16);
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        uint8_t* arow = smem + OFF_A + a * A_BYTES + r * 128;
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)  // +32 bytes along K inside the swizzled row
-          tc::mma_f16_ss(tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
-        tc::mma_commit(bar_empty + 8 * s);
+        for (int i = 0; i < 4; ++i) {
+          const int j = 4 * h + i;  // logical 16-byte chunk (8 fp16) within the 128-byte row
+          *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = dequant8(words[i], c1024z, s2);
+        }
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_aready + 8 * a);
       }
-      tc::mma_commit(bar_tmem);  // fires when every MMA above has completed
     }
-  } else if (warp >= 4) {
-    // ---------------- dequantisers, then epilogue ----------------
-    const int t = threadIdx.x - 128;     // 0..255
-    const int r = t & (BM - 1);          // weight row within the tile
-    const int h = t >> 7;                // which 32 of the k-block's 64
-    const int n = min(n0 + r, M.N - 1);  // rows past N are computed but never stored
-    const int G = M.K / kGroup;
-    const uint16_t* srow = M.scale + (size_t)n * G;
-    const uint16_t* zrow = M.zero + (size_t)n * G;
-    uint32_t c1024z = 0, s2 = 0;
-    for (int kb = 0; kb < nkb && !timed_out; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if ((kb & 1) == 0) {  // a 128-wide group spans two k-blocks
-        const __half z = __ushort_as_half(ld_u16(zrow + kb / 2));
-        const __half sc = __ushort_as_half(ld_u16(srow + kb / 2));
-        c1024z = pack_h2(__hadd(z, __float2half(1024.f)));
-        s2 = pack_h2(sc);
-      }
-      if (!tc::mbar_wait(bar_full + 8 * s, ph)) { timed_out = true; break; }
-      const uint4 cw = *reinterpret_cast<const uint4*>(smem + OFF_C + s * C_BYTES + r * 32 + h * 16);
-      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-      uint8_t* arow = smem + OFF_A + s * A_BYTES + r * 128;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int j = 4 * h + i;  // logical 16-byte chunk (8 fp16) within the 128-byte row
-        *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = dequant8(words[i], c1024z, s2);
-      }
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar_aready + 8 * s);
-    }
-    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31, tokens [half*128, half*128+128)
-    if (!timed_out) {
-      if (!tc::mbar_wait(bar_tmem, 0)) timed_out = true;
-    }
-    if (!timed_out) {
+  } else if (warp < 4) {
+    // epilogue: this warp's 32 weight rows, all bn tokens of the tile
+    int lt = 0;
+    for (int tile = t_lo; tile < t_hi && !timed_out; ++tile, ++lt) {
+      const TileInfo ti = tile_info(P, tile, mi);
+      const TcMat& M = P.m[ti.mi];
+      const int b = lt & 1;
+      if (!tc::mbar_wait(bar_tfull + 8 * b, (lt >> 1) & 1)) { timed_out = true; break; }
       tc::tc_fence_after();
-      const int q = warp & 3, half = (warp - 4) >> 2;
-      const int row = n0 + 32 * q + lane;
-      for (int c0 = half * 128; c0 < half * 128 + 128 && c0 < BN; c0 += 32) {
+      const int row = ti.n0 + 32 * warp + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(b * kTcMaxBN);
+      for (int c0 = 0; c0 < ti.bn; c0 += 32) {
         uint32_t v[32];
-        tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+        tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c0, v);
         tc::tmem_wait_ld();
         if (row < M.N) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const int m = m0 + c0 + c;
+            const int m = ti.m0 + c0 + c;
             if (m < M.M)
               M.y[(size_t)m * M.ldy + row] = __half_as_ushort(__float2half_rn(__uint_as_float(v[c])));
           }
         }
       }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_tempty + 8 * b);
     }
   }
 
@@ -224,16 +310,18 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     atomicOr(&g_device_errors, tc::kErrTimeout);
     misc[1] = 1;
   }
-  // The producer waits (bounded) for its own TMA loads still in flight before the shared
-  // memory they target is released.
-  if (warp == 0 && lane == 0 && misc[1]) {
-    for (int kb = 0; kb < issued; ++kb) tc::mbar_wait(bar_full + 8 * (kb % STAGES), (kb / STAGES) & 1);
+  __syncthreads();
+  // On the error path the producer waits (bounded) for its TMA loads that may still be in
+  // flight (the last STAGES issued) before the shared memory they target is released.
+  if (misc[1] && warp == PRODUCER_WARP && lane == 0) {
+    for (int j = (it > TSTAGES ? it - TSTAGES : 0); j < it; ++j)
+      tc::mbar_wait(bar_full + 8 * (j % TSTAGES), (j / TSTAGES) & 1);
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, kTcMaxBN);
+    tc::tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -293,6 +381,7 @@ bool tc_plan_mat(TcMat& t, const uint16_t* X, int M, const void* codes, const ui
   t.bn = bn;
   t.tiles_n = (N + BM - 1) / BM;
   t.tiles_m = (M + bn - 1) / bn;
+  t.tile_cost = K / BK + 4;  // k-blocks of the main loop + an allowance for the epilogue
   return true;
 }
 
@@ -309,7 +398,14 @@ cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  gemm_tc_int4_kernel<<<p.total_tiles, THREADS, smem, stream>>>(p);
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+  gemm_tc_int4_kernel<<<grid, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

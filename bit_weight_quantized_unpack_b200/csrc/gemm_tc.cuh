@@ -19,11 +19,13 @@ struct TcMat {
   const uint16_t* scale;
   const uint16_t* zero;
   uint16_t* y;             // fp16 [M, ldy]
-  int N, K, M, ldy, bn, tiles_n, tiles_m, tile_begin, tile_end;
+  int64_t cost_begin;      // cost of all tiles of the launch before this matrix's first
+  int N, K, M, ldy, bn, tiles_n, tiles_m, tile_begin, tile_end, tile_cost;
 };
 
 struct TcParams {
   TcMat m[kTcMaxMats];
+  int64_t total_cost;
   int count;
   int total_tiles;
 };

@@ -105,8 +105,13 @@ __device__ __forceinline__ void chunk_int2(const uint4 w, const uint16_t* const*
 
 // ---- the persistent set kernel -------------------------------------------------------
 
+// Resident CTAs per SM asked of the compiler for the batch-1 variants (register budget).
+#ifndef WQ_GEMV_MIN_BLOCKS
+#define WQ_GEMV_MIN_BLOCKS 2
+#endif
+
 template <int BITS, int MT>
-__global__ void __launch_bounds__(kGemvThreads) gemv_int_set_kernel(const __grid_constant__ SetParams P) {
+__global__ void __launch_bounds__(kGemvThreads, MT == 1 ? WQ_GEMV_MIN_BLOCKS : 1) gemv_int_set_kernel(const __grid_constant__ SetParams P) {
   const int lane = threadIdx.x & 31;
   const int warps_total = gridDim.x * (kGemvThreads / 32);
   int mi = 0;
@@ -135,47 +140,52 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int_set_kernel(const __grid
         const uint4* crow = reinterpret_cast<const uint4*>(M.codes) + (size_t)n * cpr;
         const uint16_t* srow = M.scale + (size_t)n * G;
         const uint16_t* zrow = M.zero + (size_t)n * G;
-        int c = sub;
-        // four chunks in flight per lane, then the ragged remainder
-        for (; c + 3 * L < cpr; c += 4 * L) {
-          uint4 w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) w[u] = ld_stream_v4(crow + c + u * L);
+        // This lane's chunks are sub, sub + L, sub + 2L, ... (nc of them). Two register
+        // batches of four chunks (codes + the group's scale and zero) alternate: the next
+        // batch's loads are issued before the current batch is computed, so every warp
+        // keeps four 16-byte loads in flight while it does arithmetic.
+        const int nc = (cpr - sub + L - 1) >> L2;
+        constexpr int CPG = kGroup * BITS / 128;  // 16-byte chunks per group
+        uint4 w0[4], w1[4];
+        uint16_t s0[4], s1[4], z0[4], z1[4];
+        auto load4 = [&](uint4 (&w)[4], uint16_t (&sb)[4], uint16_t (&zb)[4], int j0) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int cc = c + u * L;
-            const int g = cc / (kGroup * BITS / 128);
-            const float s = __half2float(__ushort_as_half(ld_u16(srow + g)));
-            const __half z = __ushort_as_half(ld_u16(zrow + g));
-            if (BITS == 4) {
-              const uint32_t c1 = pack_h2(__hadd(z, __float2half(1024.f)));
-              const uint32_t c16 = pack_h2(__hfma(z, __float2half(16.f), __float2half(1024.f)));
-              chunk_int4<MT>(w[u], xs, cc * 32, c1, c16, s, acc);
-            } else {
-              uint32_t cz[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                cz[j] = pack_h2(__hfma(z, __float2half((float)(1 << (2 * j))), __float2half(1024.f)));
-              chunk_int2<MT>(w[u], xs, cc * 64, cz, s, acc);
+            if (j0 + u < nc) {
+              const int cc = sub + (j0 + u) * L;
+              w[u] = ld_stream_v4(crow + cc);
+              sb[u] = ld_u16(srow + cc / CPG);
+              zb[u] = ld_u16(zrow + cc / CPG);
             }
           }
-        }
-        for (; c < cpr; c += L) {
-          const uint4 w = ld_stream_v4(crow + c);
-          const int g = c / (kGroup * BITS / 128);
-          const float s = __half2float(__ushort_as_half(ld_u16(srow + g)));
-          const __half z = __ushort_as_half(ld_u16(zrow + g));
-          if (BITS == 4) {
-            const uint32_t c1 = pack_h2(__hadd(z, __float2half(1024.f)));
-            const uint32_t c16 = pack_h2(__hfma(z, __float2half(16.f), __float2half(1024.f)));
-            chunk_int4<MT>(w, xs, c * 32, c1, c16, s, acc);
-          } else {
-            uint32_t cz[4];
+        };
+        auto run4 = [&](const uint4 (&w)[4], const uint16_t (&sb)[4], const uint16_t (&zb)[4], int j0) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              cz[j] = pack_h2(__hfma(z, __float2half((float)(1 << (2 * j))), __float2half(1024.f)));
-            chunk_int2<MT>(w, xs, c * 64, cz, s, acc);
+          for (int u = 0; u < 4; ++u) {
+            if (j0 + u < nc) {
+              const int cc = sub + (j0 + u) * L;
+              const float sf = __half2float(__ushort_as_half(sb[u]));
+              const __half z = __ushort_as_half(zb[u]);
+              if (BITS == 4) {
+                const uint32_t c1 = pack_h2(__hadd(z, __float2half(1024.f)));
+                const uint32_t c16 = pack_h2(__hfma(z, __float2half(16.f), __float2half(1024.f)));
+                chunk_int4<MT>(w[u], xs, cc * 32, c1, c16, sf, acc);
+              } else {
+                uint32_t cz[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  cz[j] = pack_h2(__hfma(z, __float2half((float)(1 << (2 * j))), __float2half(1024.f)));
+                chunk_int2<MT>(w[u], xs, cc * 64, cz, sf, acc);
+              }
+            }
           }
+        };
+        load4(w0, s0, z0, 0);
+        for (int j0 = 0; j0 < nc; j0 += 8) {
+          load4(w1, s1, z1, j0 + 4);
+          run4(w0, s0, z0, j0);
+          load4(w0, s0, z0, j0 + 8);
+          run4(w1, s1, z1, j0 + 4);
         }
       }
       // split-K reduction over the L lanes of a row (warp shuffles), then one fp16 store

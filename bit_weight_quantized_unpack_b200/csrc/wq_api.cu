@@ -40,6 +40,10 @@ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0;
 
 constexpr int64_t kMaxK = (int64_t)1 << 20;
 
+// Which matrix-vector kernel serves batch 1: the register-streaming kernel (gemv.cu) or
+// the bulk-copy-staged one (gemv_bulk.cu). Both compute identical results.
+constexpr bool kUseBulkGemv = false;
+
 int check_shape(int fmt, int64_t N, int64_t K) {
   if (fmt < WQ_INT4 || fmt > WQ_TERNARY) return WQ_ERR_ARG;
   if (N < 1 || N > INT_MAX || K < 128 || K > kMaxK || K % 128 != 0) return WQ_ERR_SHAPE;
@@ -142,11 +146,13 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
       return WQ_ERR_CUDA;
     tp.m[0].tile_begin = 0;
     tp.m[0].tile_end = tp.m[0].tiles_n * tp.m[0].tiles_m;
+    tp.m[0].cost_begin = 0;
     tp.count = 1;
     tp.total_tiles = tp.m[0].tile_end;
+    tp.total_cost = (int64_t)tp.total_tiles * tp.m[0].tile_cost;
     return cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
   }
-  if (M == 1 && fmt != WQ_TERNARY) {
+  if (M == 1 && fmt != WQ_TERNARY && kUseBulkGemv) {
     static thread_local wq::BulkParams bp;
     const wq_linear_desc d = {codes, scale, zero, X, Y, N, K};
     if (plan_bulk(bp, fmt, 1, &d)) return cuda_status(wq::launch_gemv_bulk(bp, fmt == WQ_INT4 ? 4 : 2, (cudaStream_t)stream));
@@ -187,7 +193,7 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   }
   int st0 = check_device();
   if (st0 != WQ_OK) return st0;
-  {
+  if (kUseBulkGemv) {
     static thread_local wq::BulkParams bp;
     if (plan_bulk(bp, fmt, count, descs))
       return cuda_status(wq::launch_gemv_bulk(bp, fmt == WQ_INT4 ? 4 : 2, (cudaStream_t)stream));
