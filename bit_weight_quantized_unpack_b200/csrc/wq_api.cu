@@ -6,6 +6,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_bulk.cuh"
+#include "gemv_rows.cuh"
 #include "wq.h"
 
 namespace {
@@ -102,6 +103,23 @@ bool plan_bulk(wq::BulkParams& p, int fmt, int count, const wq_linear_desc* d) {
   return true;
 }
 
+// Row-per-lane kernel for a batch-1 set (int4 / int2): needs 32-byte aligned codes
+// (its loads are whole 32-byte sectors) and K small enough to stage x in shared memory.
+int try_rows(int fmt, int count, const wq_linear_desc* d, cudaStream_t stream, bool* done) {
+  *done = false;
+  if (fmt == WQ_TERNARY || count > wq::kRowsMaxMats) return WQ_OK;
+  static thread_local wq::RowParams rp;
+  static thread_local wq::RowMatDesc rd[wq::kRowsMaxMats];
+  for (int i = 0; i < count; ++i) {
+    if (((uintptr_t)d[i].codes & 31) != 0) return WQ_OK;
+    rd[i] = {d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K};
+  }
+  int max_k = 0;
+  if (!wq::rows_plan(rp, fmt == WQ_INT4 ? 4 : 2, count, rd, &max_k)) return WQ_OK;
+  *done = true;
+  return cuda_status(wq::launch_gemv_rows(rp, fmt == WQ_INT4 ? 4 : 2, max_k, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -152,6 +170,12 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
     tp.total_cost = (int64_t)tp.total_tiles * tp.m[0].tile_cost;
     return cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
   }
+  if (M == 1) {
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K};
+    bool done = false;
+    const int r = try_rows(fmt, 1, &d, (cudaStream_t)stream, &done);
+    if (done) return r;
+  }
   if (M == 1 && fmt != WQ_TERNARY && kUseBulkGemv) {
     static thread_local wq::BulkParams bp;
     const wq_linear_desc d = {codes, scale, zero, X, Y, N, K};
@@ -193,6 +217,11 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   }
   int st0 = check_device();
   if (st0 != WQ_OK) return st0;
+  {
+    bool done = false;
+    const int r = try_rows(fmt, count, descs, (cudaStream_t)stream, &done);
+    if (done) return r;
+  }
   if (kUseBulkGemv) {
     static thread_local wq::BulkParams bp;
     if (plan_bulk(bp, fmt, count, descs))
