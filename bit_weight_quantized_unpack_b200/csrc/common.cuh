@@ -63,6 +63,11 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t v, uint32_t mask, uint32
 }  // namespace wq
 
 namespace wq {
+__device__ __forceinline__ uint32_t prmt_u32(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
 __device__ __forceinline__ uint32_t pack_h2(__half h) {
   const uint32_t b = __half_as_ushort(h);
   return b | (b << 16);

@@ -36,22 +36,33 @@ namespace {
 
 constexpr int BM = 128;       // weight rows per tile
 constexpr int BK = 64;        // k per stage: one 128-byte swizzle row of fp16
-constexpr int TSTAGES = 5;    // TMA ring: activation tile + codes of one k-block
+constexpr int XSTAGES = 4;    // activation tiles [bn x 64] (read from L2)
+constexpr int CRING = 12;     // per-thread ring of code chunks: 11 k-blocks in flight
 constexpr int ASTAGES = 2;    // dequantised weight tiles (written by CUDA cores, read by MMA)
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB of dequantised fp16 weights
 constexpr int B_BYTES = kTcMaxBN * BK * 2;      // 32 KB of activations
-constexpr int C_BYTES = BM * BK / 2;            // 4 KB of int4 codes
-constexpr int T_BYTES = B_BYTES + C_BYTES;      // one TMA stage
+constexpr int CR_BYTES = BM * BK / 2;          // 4 KB of int4 codes per k-block
 constexpr int OFF_A = 0;
-constexpr int OFF_T = OFF_A + ASTAGES * A_BYTES;
-constexpr int OFF_BAR = OFF_T + TSTAGES * T_BYTES;
-constexpr int NUM_BARS = 2 * TSTAGES + 2 * ASTAGES + 4;
+constexpr int OFF_X = OFF_A + ASTAGES * A_BYTES;
+constexpr int OFF_C = OFF_X + XSTAGES * B_BYTES;
+constexpr int EPI_BYTES = 32 * 32 * 2;          // one warp's 32 x 32 fp16 output block
+constexpr int OFF_E = OFF_C + CRING * CR_BYTES;  // [4 warps][2 buffers] staged output blocks
+constexpr int OFF_BAR = OFF_E + 4 * 2 * EPI_BYTES;
+constexpr int NUM_BARS = 2 * XSTAGES + 2 * ASTAGES + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
 constexpr int THREADS = 512;                    // 16 warps
-constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, DEQ_WARP0 = 8, DEQ_WARPS = 8;
+constexpr int XPROD_WARP = 4, MMA_WARP = 5, DEQ_WARP0 = 8, DEQ_WARPS = 8;
 constexpr int TMEM_COLS = 2 * kTcMaxBN;         // two accumulator buffers
-static_assert(T_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzled operands need 1 KB alignment");
+static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled operands need 1 KB alignment");
+
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_ring() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(CRING - 1) : "memory");
+}
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
@@ -82,7 +93,8 @@ __device__ __forceinline__ uint4 dequant8(uint32_t v, uint32_t c1024z, uint32_t 
 }
 
 // First tile whose starting cost is >= target (tiles of all matrices numbered in order).
-__device__ int first_tile_at(const TcParams& P, int64_t target) {
+template <int CAP>
+__device__ int first_tile_at(const TcParamsT<CAP>& P, int64_t target) {
   for (int i = 0; i < P.count; ++i) {
     const TcMat& m = P.m[i];
     const int64_t end = m.cost_begin + (int64_t)(m.tile_end - m.tile_begin) * m.tile_cost;
@@ -99,7 +111,8 @@ struct TileInfo {
   int mi, n0, m0, bn, nkb;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const TcParams& P, int tile, int& mi) {
+template <int CAP>
+__device__ __forceinline__ TileInfo tile_info(const TcParamsT<CAP>& P, int tile, int& mi) {
   while (tile >= P.m[mi].tile_end) ++mi;
   const TcMat& M = P.m[mi];
   const int local = tile - M.tile_begin;
@@ -119,14 +132,15 @@ __device__ __forceinline__ TileInfo tile_info(const TcParams& P, int tile, int& 
 // 5 MMA issuer (and TMEM owner), 8-15 dequantisers (two threads per weight row, 32 k each
 // per stage); 6-7 idle. The two 256-column TMEM accumulators let the epilogue of one tile
 // overlap the main loop of the next.
-__global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_constant__ TcParams P) {
+template <int CAP>
+__global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_constant__ TcParamsT<CAP> P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment of the operand buffers is what the 128-byte swizzle assumes
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = tc::smem_u32(smem);
-  const uint32_t bar_full = sbase + OFF_BAR;                  // [TSTAGES] TMA: X tile + codes landed
-  const uint32_t bar_empty = bar_full + 8 * TSTAGES;          // [TSTAGES] MMAs reading it done
-  const uint32_t bar_aready = bar_empty + 8 * TSTAGES;        // [ASTAGES] dequantised A written
+  const uint32_t bar_xfull = sbase + OFF_BAR;                 // [XSTAGES] activation tile landed
+  const uint32_t bar_xempty = bar_xfull + 8 * XSTAGES;        // [XSTAGES] MMAs reading it done
+  const uint32_t bar_aready = bar_xempty + 8 * XSTAGES;       // [ASTAGES] dequantised A written
   const uint32_t bar_aempty = bar_aready + 8 * ASTAGES;       // [ASTAGES] MMAs reading A done
   const uint32_t bar_tfull = bar_aempty + 8 * ASTAGES;        // [2] accumulator complete
   const uint32_t bar_tempty = bar_tfull + 16;                 // [2] accumulator drained
@@ -135,9 +149,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < TSTAGES; ++i) {
-      tc::mbar_init(bar_full + 8 * i, 1);
-      tc::mbar_init(bar_empty + 8 * i, 1);
+    for (int i = 0; i < XSTAGES; ++i) {
+      tc::mbar_init(bar_xfull + 8 * i, 1);
+      tc::mbar_init(bar_xempty + 8 * i, 1);
     }
     for (int i = 0; i < ASTAGES; ++i) {
       tc::mbar_init(bar_aready + 8 * i, DEQ_WARPS);
@@ -164,23 +178,22 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   const int t_hi = first_tile_at(P, share * (blockIdx.x + 1));
 
   bool timed_out = false;
-  int it = 0;  // k-block sequence number over this CTA's tiles
+  int it = 0;    // k-block sequence number over this CTA's tiles
   int mi = 0;
 
-  if (warp == PRODUCER_WARP) {
+  if (warp == XPROD_WARP) {
+    // activation tiles, one per k-block
     if (lane == 0) {
       for (int tile = t_lo; tile < t_hi && !timed_out; ++tile) {
         const TileInfo ti = tile_info(P, tile, mi);
         const TcMat& M = P.m[ti.mi];
-        const uint32_t tx = (uint32_t)(ti.bn * BK * 2 + C_BYTES);
+        const uint32_t tx = (uint32_t)(ti.bn * BK * 2);
         for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-          const int s = it % TSTAGES;
-          if (!tc::mbar_wait(bar_empty + 8 * s, ((it / TSTAGES) & 1) ^ 1)) { timed_out = true; break; }
+          const int s = it % XSTAGES;
+          if (!tc::mbar_wait(bar_xempty + 8 * s, ((it / XSTAGES) & 1) ^ 1)) { timed_out = true; break; }
           if (misc[1]) { timed_out = true; break; }
-          const uint32_t st = sbase + OFF_T + s * T_BYTES;
-          tc::mbar_arrive_expect_tx(bar_full + 8 * s, tx);
-          tc::tma_load_2d(st, &M.tmap_x, bar_full + 8 * s, kb * BK, ti.m0);
-          tc::tma_load_2d(st + B_BYTES, &M.tmap_codes, bar_full + 8 * s, kb * (BK / 2), ti.n0);
+          tc::mbar_arrive_expect_tx(bar_xfull + 8 * s, tx);
+          tc::tma_load_2d(sbase + OFF_X + s * B_BYTES, &M.tmap_x, bar_xfull + 8 * s, kb * BK, ti.m0);
         }
       }
     }
@@ -195,19 +208,19 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
         const uint32_t d_tmem = tmem + (uint32_t)(b * kTcMaxBN);
         const uint32_t idesc = tc::idesc_f16_f32(BM, ti.bn);
         for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-          const int s = it % TSTAGES, a = it % ASTAGES;
-          if (!tc::mbar_wait(bar_full + 8 * s, (it / TSTAGES) & 1) ||
+          const int s = it % XSTAGES, a = it % ASTAGES;
+          if (!tc::mbar_wait(bar_xfull + 8 * s, (it / XSTAGES) & 1) ||
               !tc::mbar_wait(bar_aready + 8 * a, (it / ASTAGES) & 1)) {
             timed_out = true;
             break;
           }
           tc::tc_fence_after();
           const uint64_t ad = tc::sw128_kmajor_desc(sbase + OFF_A + a * A_BYTES);
-          const uint64_t bd = tc::sw128_kmajor_desc(sbase + OFF_T + s * T_BYTES);
+          const uint64_t bd = tc::sw128_kmajor_desc(sbase + OFF_X + s * B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)  // +32 bytes along K inside the swizzled row
             tc::mma_f16_ss(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
-          tc::mma_commit(bar_empty + 8 * s);   // frees the TMA stage ...
+          tc::mma_commit(bar_xempty + 8 * s);  // frees the activation stage ...
           tc::mma_commit(bar_aempty + 8 * a);  // ... and the dequantised tile
         }
         tc::mma_commit(bar_tfull + 8 * b);  // fires when every MMA of the tile has completed
@@ -223,6 +236,30 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
       const int G = M.K / kGroup;
       return (uint32_t)ld_u16(M.scale + (size_t)n * G + g) | ((uint32_t)ld_u16(M.zero + (size_t)n * G + g) << 16);
     };
+    // Codes are not copied by TMA: a slow DRAM copy would hold up the activation copies
+    // queued behind it. Each thread streams its own 16-byte chunk of every k-block of its
+    // row with cp.async into its slot of a CRING-deep ring ([slot][thread] x 16 bytes),
+    // CRING - 1 k-blocks ahead, across tile boundaries.
+    const uint32_t cring = sbase + OFF_C + 16u * (uint32_t)t;
+    int f_tile = t_lo, f_kb = 0, f_mi = 0, fseq = 0;
+    TileInfo f_ti{};
+    if (f_tile < t_hi) f_ti = tile_info(P, f_tile, f_mi);
+    auto fetch_next = [&]() {
+      if (f_tile < t_hi) {
+        const TcMat& Mf = P.m[f_ti.mi];
+        const int nf = min(f_ti.n0 + r, Mf.N - 1);
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(Mf.codes) + (size_t)nf * (Mf.K / 2) + f_kb * (BK / 2) + h * 16;
+        cp_async16(cring + (uint32_t)(fseq % CRING) * (CR_BYTES), src);
+        if (++f_kb == f_ti.nkb) {
+          f_kb = 0;
+          if (++f_tile < t_hi) f_ti = tile_info(P, f_tile, f_mi);
+        }
+      }
+      cp_async_commit();
+      ++fseq;
+    };
+    for (int i = 0; i < CRING - 1; ++i) fetch_next();
+    int cseq = 0;
     uint32_t pre0 = 0, pre1 = 0;
     int mi_pre = 0;
     if (t_lo < t_hi) {
@@ -241,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
       uint32_t c1024z = 0, s2 = 0;
       const int kb_pre = ti.nkb > 4 ? ti.nkb - 4 : 0;
       for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-        const int s = it % TSTAGES, a = it % ASTAGES;
+        const int a = it % ASTAGES;
         if ((kb & 1) == 0) {
           const int g = kb >> 1;
           if (g + 2 < G) sz2 = load_sz(M, n, g + 2);
@@ -258,12 +295,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
           pre0 = load_sz(Mn, nn, 0);
           pre1 = Mn.K > kGroup ? load_sz(Mn, nn, 1) : 0u;
         }
-        if (!tc::mbar_wait(bar_full + 8 * s, (it / TSTAGES) & 1) ||
-            !tc::mbar_wait(bar_aempty + 8 * a, ((it / ASTAGES) & 1) ^ 1)) {
-          timed_out = true;
-          break;
-        }
-        const uint4 cw = *reinterpret_cast<const uint4*>(smem + OFF_T + s * T_BYTES + B_BYTES + r * 32 + h * 16);
+        fetch_next();
+        cp_async_wait_ring();  // this k-block's chunk (issued CRING - 1 fetches ago) has landed
+        if (!tc::mbar_wait(bar_aempty + 8 * a, ((it / ASTAGES) & 1) ^ 1)) { timed_out = true; break; }
+        const uint4 cw = *reinterpret_cast<const uint4*>(smem + OFF_C + (cseq % CRING) * CR_BYTES + 16 * t);
+        ++cseq;
         const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
         uint8_t* arow = smem + OFF_A + a * A_BYTES + r * 128;
 #pragma unroll
@@ -276,9 +312,15 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
         if (lane == 0) tc::mbar_arrive(bar_aready + 8 * a);
       }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp < 4) {
-    // epilogue: this warp's 32 weight rows, all bn tokens of the tile
-    int lt = 0;
+    // epilogue: this warp's 32 weight rows, all bn tokens of the tile. Each 32-token block
+    // is transposed through shared memory into Y's [token][row] order and written by one
+    // TMA tensor store; per-thread 2-byte global stores would flood the SM's memory path
+    // and delay the TMA loads queued behind them.
+    int lt = 0, nst = 0;
+    const uint32_t ebuf = sbase + OFF_E + (uint32_t)(warp * 2 * EPI_BYTES);
+    uint16_t* ebuf_g = reinterpret_cast<uint16_t*>(smem + OFF_E + warp * 2 * EPI_BYTES);
     for (int tile = t_lo; tile < t_hi && !timed_out; ++tile, ++lt) {
       const TileInfo ti = tile_info(P, tile, mi);
       const TcMat& M = P.m[ti.mi];
@@ -287,11 +329,24 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
       tc::tc_fence_after();
       const int row = ti.n0 + 32 * warp + lane;
       const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(b * kTcMaxBN);
-      for (int c0 = 0; c0 < ti.bn; c0 += 32) {
+      for (int c0 = 0; c0 < ti.bn; c0 += 32, ++nst) {
         uint32_t v[32];
         tc::tmem_ld_32x32b_x32(taddr + (uint32_t)c0, v);
         tc::tmem_wait_ld();
-        if (row < M.N) {
+        if (M.y_tma) {
+          // staging buffer nst & 1: the store issued from it two blocks ago has read it
+          if (lane == 0) tc::bulk_wait_read<1>();
+          __syncwarp();
+          uint16_t* eb = ebuf_g + (nst & 1) * (EPI_BYTES / 2);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) eb[c * 32 + lane] = __half_as_ushort(__float2half_rn(__uint_as_float(v[c])));
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_store_2d(&M.tmap_y, ebuf + (uint32_t)((nst & 1) * EPI_BYTES), ti.n0 + 32 * warp, ti.m0 + c0);
+            tc::bulk_commit();
+          }
+        } else if (row < M.N) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int m = ti.m0 + c0 + c;
@@ -304,6 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(bar_tempty + 8 * b);
     }
+    if (lane == 0) tc::bulk_wait_all();  // stores complete before the kernel exits
   }
 
   if (timed_out) {
@@ -311,11 +367,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     misc[1] = 1;
   }
   __syncthreads();
-  // On the error path the producer waits (bounded) for its TMA loads that may still be in
-  // flight (the last STAGES issued) before the shared memory they target is released.
-  if (misc[1] && warp == PRODUCER_WARP && lane == 0) {
-    for (int j = (it > TSTAGES ? it - TSTAGES : 0); j < it; ++j)
-      tc::mbar_wait(bar_full + 8 * (j % TSTAGES), (j / TSTAGES) & 1);
+  // On the error path each producer waits (bounded) for its own TMA loads that may still be
+  // in flight before the shared memory they target is released.
+  if (misc[1] && lane == 0) {
+    if (warp == XPROD_WARP)
+      for (int j = (it > XSTAGES ? it - XSTAGES : 0); j < it; ++j)
+        tc::mbar_wait(bar_xfull + 8 * (j % XSTAGES), (j / XSTAGES) & 1);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -361,16 +418,20 @@ bool tc_plan_mat(TcMat& t, const uint16_t* X, int M, const void* codes, const ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)N};
-    const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
-    const cuuint32_t box[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)BM};
+  // Y [M, N] fp16 as a tensor for the epilogue's TMA stores (box 32 rows x 32 tokens);
+  // needs N * 2 bytes a multiple of 16 and a 16-byte aligned base, else plain stores
+  t.y_tma = 0;
+  if (N % 8 == 0 && ((uintptr_t)Y & 15) == 0) {
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    const cuuint32_t box[2] = {32, 32};
     const cuuint32_t es[2] = {1, 1};
-    if (enc(&t.tmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
+    if (enc(&t.tmap_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Y, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      t.y_tma = 1;
   }
+  t.codes = codes;
   t.scale = scale;
   t.zero = zero;
   t.y = Y;
@@ -390,11 +451,12 @@ int tc_bn_for(int M) {
   return bn < kTcMaxBN ? bn : kTcMaxBN;
 }
 
-cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream) {
+template <int CAP>
+static cudaError_t launch_cap(const TcParamsT<CAP>& p, cudaStream_t stream) {
   static bool attr = false;
   const int smem = SMEM_USED + 1024;  // + alignment slack
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_int4_kernel<CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -405,8 +467,20 @@ cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-  gemm_tc_int4_kernel<<<grid, THREADS, smem, stream>>>(p);
+  gemm_tc_int4_kernel<CAP><<<grid, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream) {
+  if (p.count == 1) {
+    TcParamsT<1> p1;
+    p1.m[0] = p.m[0];
+    p1.total_cost = p.total_cost;
+    p1.count = 1;
+    p1.total_tiles = p.total_tiles;
+    return launch_cap<1>(p1, stream);
+  }
+  return launch_cap<kTcMaxMats>(p, stream);
 }
 
 unsigned int* device_error_word() {

@@ -8,27 +8,32 @@
 namespace wq {
 
 constexpr int kTcMaxBN = 256;   // tokens per tile (MMA N), also the TMEM columns allocated
-constexpr int kTcMaxMats = 64;  // matrices per launch (tensor maps travel as kernel params)
+constexpr int kTcMaxMats = 48;  // matrices per launch (tensor maps travel as kernel params)
 constexpr int kTcMinM = 16;     // wq_gemm uses the tensor-core path from this M up (int4)
 
 // One matrix: tiles [tile_begin, tile_end) of the launch, tiles_m token tiles per
 // 128-row weight tile. Tensor maps first: CUtensorMap needs 64-byte alignment.
 struct TcMat {
   CUtensorMap tmap_x;      // X [M, K] fp16, box 64 x bn, 128-byte swizzle
-  CUtensorMap tmap_codes;  // int4 codes as bytes [N, K/2], box 32 x 128
+  CUtensorMap tmap_y;      // Y [M, N] fp16, box 32 x 32 (valid when y_tma)
+  const void* codes;       // int4 codes uint32 [N, K/8] (streamed with cp.async, not TMA)
   const uint16_t* scale;
   const uint16_t* zero;
   uint16_t* y;             // fp16 [M, ldy]
   int64_t cost_begin;      // cost of all tiles of the launch before this matrix's first
   int N, K, M, ldy, bn, tiles_n, tiles_m, tile_begin, tile_end, tile_cost;
+  int y_tma;               // the epilogue stores Y through tmap_y
 };
 
-struct TcParams {
-  TcMat m[kTcMaxMats];
+// Passed by value as the kernel parameter; CAP is chosen per call (1 for a single matrix).
+template <int CAP>
+struct TcParamsT {
+  TcMat m[CAP];
   int64_t total_cost;
   int count;
   int total_tiles;
 };
+using TcParams = TcParamsT<kTcMaxMats>;
 
 bool tc_plan_mat(TcMat& t, const uint16_t* X, int M, const void* codes, const uint16_t* scale,
                  const uint16_t* zero, uint16_t* Y, int N, int K, int bn);

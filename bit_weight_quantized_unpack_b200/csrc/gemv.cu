@@ -110,8 +110,8 @@ __device__ __forceinline__ void chunk_int2(const uint4 w, const uint16_t* const*
 #define WQ_GEMV_MIN_BLOCKS 2
 #endif
 
-template <int BITS, int MT>
-__global__ void __launch_bounds__(kGemvThreads, MT == 1 ? WQ_GEMV_MIN_BLOCKS : 1) gemv_int_set_kernel(const __grid_constant__ SetParams P) {
+template <int BITS, int MT, int CAP>
+__global__ void __launch_bounds__(kGemvThreads, MT == 1 ? WQ_GEMV_MIN_BLOCKS : 1) gemv_int_set_kernel(const __grid_constant__ SetParamsT<CAP> P) {
   const int lane = threadIdx.x & 31;
   const int warps_total = gridDim.x * (kGemvThreads / 32);
   int mi = 0;
@@ -204,8 +204,8 @@ __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? WQ_GEMV_MIN_BLOCKS : 1
 
 // ---- ternary (first version: per-byte base-3 digit extraction) ----------------------
 
-template <int MT>
-__global__ void __launch_bounds__(kGemvThreads) gemv_ternary_set_kernel(const __grid_constant__ SetParams P) {
+template <int MT, int CAP>
+__global__ void __launch_bounds__(kGemvThreads) gemv_ternary_set_kernel(const __grid_constant__ SetParamsT<CAP> P) {
   const int lane = threadIdx.x & 31;
   const int warps_total = gridDim.x * (kGemvThreads / 32);
   int mi = 0;
@@ -279,25 +279,37 @@ static int grid_for(const void* kernel, int total_items) {
   return need < sms * per_sm ? need : sms * per_sm;
 }
 
-template <int BITS, int MT>
-static cudaError_t launch_int(const SetParams& p, cudaStream_t stream) {
-  const void* k = (const void*)gemv_int_set_kernel<BITS, MT>;
-  gemv_int_set_kernel<BITS, MT><<<grid_for(k, p.total_items), kGemvThreads, 0, stream>>>(p);
+template <int BITS, int MT, int CAP>
+static cudaError_t launch_int(const SetParamsT<CAP>& p, cudaStream_t stream) {
+  const void* k = (const void*)gemv_int_set_kernel<BITS, MT, CAP>;
+  gemv_int_set_kernel<BITS, MT, CAP><<<grid_for(k, p.total_items), kGemvThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <int MT>
-static cudaError_t launch_ternary(const SetParams& p, cudaStream_t stream) {
-  const void* k = (const void*)gemv_ternary_set_kernel<MT>;
-  gemv_ternary_set_kernel<MT><<<grid_for(k, p.total_items), kGemvThreads, 0, stream>>>(p);
+template <int MT, int CAP>
+static cudaError_t launch_ternary(const SetParamsT<CAP>& p, cudaStream_t stream) {
+  const void* k = (const void*)gemv_ternary_set_kernel<MT, CAP>;
+  gemv_ternary_set_kernel<MT, CAP><<<grid_for(k, p.total_items), kGemvThreads, 0, stream>>>(p);
   return cudaGetLastError();
+}
+
+template <int CAP>
+static cudaError_t launch_cap(const SetParamsT<CAP>& p, int fmt, int max_m, cudaStream_t stream) {
+  const bool multi = max_m > 1;
+  if (fmt == 0) return multi ? launch_int<4, 4, CAP>(p, stream) : launch_int<4, 1, CAP>(p, stream);
+  if (fmt == 1) return multi ? launch_int<2, 4, CAP>(p, stream) : launch_int<2, 1, CAP>(p, stream);
+  return multi ? launch_ternary<4, CAP>(p, stream) : launch_ternary<1, CAP>(p, stream);
 }
 
 cudaError_t launch_gemv_set(const SetParams& p, int fmt, int max_m, cudaStream_t stream) {
-  const bool multi = max_m > 1;
-  if (fmt == 0) return multi ? launch_int<4, 4>(p, stream) : launch_int<4, 1>(p, stream);
-  if (fmt == 1) return multi ? launch_int<2, 4>(p, stream) : launch_int<2, 1>(p, stream);
-  return multi ? launch_ternary<4>(p, stream) : launch_ternary<1>(p, stream);
+  if (p.count == 1) {  // a single matrix: a one-entry parameter block
+    SetParamsT<1> p1;
+    p1.count = 1;
+    p1.total_items = p.total_items;
+    p1.m[0] = p.m[0];
+    return launch_cap<1>(p1, fmt, max_m, stream);
+  }
+  return launch_cap<kSetMax>(p, fmt, max_m, stream);
 }
 
 }  // namespace wq

@@ -24,11 +24,13 @@ struct SetMat {
 
 // Passed by value as a __grid_constant__ kernel parameter (about 15 KB): the set needs
 // no device-side table and the library allocates nothing.
-struct SetParams {
+template <int CAP>
+struct SetParamsT {
   int count;
   int total_items;
-  SetMat m[kSetMax];
+  SetMat m[CAP];
 };
+using SetParams = SetParamsT<kSetMax>;
 
 int gemv_lanes_log2(int fmt, int64_t K);
 cudaError_t launch_gemv_set(const SetParams& p, int fmt, int max_m, cudaStream_t stream);

@@ -12,7 +12,7 @@
 //     multiply-add reads both of its fp16 operands from the low half of a register;
 // Work split: rows of all matrices of a set are laid end to end with their byte cost; CTA
 // b processes the rows whose first byte falls in its 1/gridDim share (so every CTA
-// streams the same number of bytes), 256 rows at a time, matrix by matrix.
+// streams the same number of bytes), matrix by matrix, its warps taking 32-row units.
 //
 // Arithmetic per 32-bit word of codes is the one of gemv.cu: binary16 magic numbers give
 // q - z exactly, each product with an fp16 activation is exact in binary32, and only the
@@ -33,16 +33,19 @@ __device__ __forceinline__ uint32_t ld_meta(const uint16_t* s, const uint16_t* z
 }
 
 // x value k of the staged activation vector as an f16 operand (low half of a word).
-template <bool XEXP>
+template <int XM>
 __device__ __forceinline__ uint16_t xval(const uint32_t* xs, int k) {
-  if (XEXP) return (uint16_t)xs[k];
+  if (XM == 0) return (uint16_t)xs[k];
   const uint32_t w = xs[k >> 1];
   return (k & 1) ? hi16(w) : lo16(w);
 }
 
 // One int4 group (128 weights = 16 words in two sectors) of a row against x[k0 .. k0+127].
 // Four accumulators (even / odd words x plain / 16x lanes) keep four independent chains.
-template <bool XEXP>
+// XM selects the staged layout of x: 0 = one fp16 per 32-bit word; 1 = fp16 pairs in
+// natural order; 2 = fp16 pairs (x_j, x_j+4) of each group of eight, matching the code
+// pairs of one word of codes, so both operands of every multiply sit in the same half.
+template <int XM>
 __device__ __forceinline__ float group_int4(const uint32_t (&c)[16], const uint32_t* xs, int k0, uint32_t sz) {
   const __half z = __ushort_as_half((uint16_t)(sz >> 16));
   const uint32_t c1 = pack_h2(__hadd(z, __float2half(1024.f)));
@@ -55,19 +58,31 @@ __device__ __forceinline__ float group_int4(const uint32_t (&c)[16], const uint3
     const uint32_t d1 = hsub2_u32(lop_and_or(v, 0x00F000F0u, 0x64006400u), c16);   // 16 q1, 16 q5
     const uint32_t d2 = hsub2_u32(lop_and_or(v8, 0x000F000Fu, 0x64006400u), c1);   // q2, q6
     const uint32_t d3 = hsub2_u32(lop_and_or(v8, 0x00F000F0u, 0x64006400u), c16);  // 16 q3, 16 q7
+    float& A = a[i & 1];
+    float& B = b[i & 1];
+    if (XM == 2) {  // one 16-byte load: (x0,x4) (x1,x5) (x2,x6) (x3,x7)
+      const uint4 w = reinterpret_cast<const uint4*>(xs + k0 / 2)[i];
+      A = fma_f16f16_f32(lo16(d0), lo16(w.x), A);
+      A = fma_f16f16_f32(hi16(d0), hi16(w.x), A);
+      A = fma_f16f16_f32(lo16(d2), lo16(w.z), A);
+      A = fma_f16f16_f32(hi16(d2), hi16(w.z), A);
+      B = fma_f16f16_f32(lo16(d1), lo16(w.y), B);
+      B = fma_f16f16_f32(hi16(d1), hi16(w.y), B);
+      B = fma_f16f16_f32(lo16(d3), lo16(w.w), B);
+      B = fma_f16f16_f32(hi16(d3), hi16(w.w), B);
+      continue;
+    }
     uint16_t x[8];
-    if (XEXP) {  // two 16-byte shared loads: x[k .. k+3], x[k+4 .. k+7], one per 32-bit word
+    if (XM == 0) {  // two 16-byte shared loads: x[k .. k+3], x[k+4 .. k+7], one per 32-bit word
       const uint4 lo = reinterpret_cast<const uint4*>(xs + k0)[2 * i];
       const uint4 hi = reinterpret_cast<const uint4*>(xs + k0)[2 * i + 1];
       x[0] = lo16(lo.x); x[1] = lo16(lo.y); x[2] = lo16(lo.z); x[3] = lo16(lo.w);
       x[4] = lo16(hi.x); x[5] = lo16(hi.y); x[6] = lo16(hi.z); x[7] = lo16(hi.w);
-    } else {     // one 16-byte shared load of four fp16x2 words
+    } else {        // one 16-byte shared load of four fp16x2 words
       const uint4 w = reinterpret_cast<const uint4*>(xs + k0 / 2)[i];
       x[0] = lo16(w.x); x[1] = hi16(w.x); x[2] = lo16(w.y); x[3] = hi16(w.y);
       x[4] = lo16(w.z); x[5] = hi16(w.z); x[6] = lo16(w.w); x[7] = hi16(w.w);
     }
-    float& A = a[i & 1];
-    float& B = b[i & 1];
     A = fma_f16f16_f32(lo16(d0), x[0], A);
     A = fma_f16f16_f32(hi16(d0), x[4], A);
     A = fma_f16f16_f32(lo16(d2), x[2], A);
@@ -81,7 +96,7 @@ __device__ __forceinline__ float group_int4(const uint32_t (&c)[16], const uint3
 }
 
 // One int2 group (128 weights = 8 words in one sector).
-template <bool XEXP>
+template <int XM>
 __device__ __forceinline__ float group_int2(const uint32_t (&c)[8], const uint32_t* xs, int k0, uint32_t sz) {
   const __half z = __ushort_as_half((uint16_t)(sz >> 16));
   constexpr uint32_t kMask[4] = {0x00030003u, 0x000C000Cu, 0x00300030u, 0x00C000C0u};
@@ -97,8 +112,8 @@ __device__ __forceinline__ float group_int2(const uint32_t (&c)[8], const uint32
     for (int j = 0; j < 8; ++j) {
       // lanes of d: codes j and j + 8 of the word, scaled by 4^(j & 3)
       const uint32_t d = hsub2_u32(lop_and_or(j < 4 ? v : v8, kMask[j & 3], 0x64006400u), cz[j & 3]);
-      a[j & 3] = fma_f16f16_f32(lo16(d), xval<XEXP>(xs, k + j), a[j & 3]);
-      a[j & 3] = fma_f16f16_f32(hi16(d), xval<XEXP>(xs, k + j + 8), a[j & 3]);
+      a[j & 3] = fma_f16f16_f32(lo16(d), xval<XM>(xs, k + j), a[j & 3]);
+      a[j & 3] = fma_f16f16_f32(hi16(d), xval<XM>(xs, k + j + 8), a[j & 3]);
     }
   }
   return fmaf(a[3], 0.015625f, fmaf(a[2], 0.0625f, fmaf(a[1], 0.25f, a[0])));
@@ -124,12 +139,15 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+#ifndef WQ_ROWS_XMODE
+#define WQ_ROWS_XMODE 1
+#endif
 #ifndef WQ_ROWS_MIN_BLOCKS
 #define WQ_ROWS_MIN_BLOCKS 3
 #endif
 
-template <int BITS, bool XEXP>
-__global__ void __launch_bounds__(THREADS, WQ_ROWS_MIN_BLOCKS) gemv_rows_kernel(const __grid_constant__ RowParams P) {
+template <int BITS, int XM, int CAP>
+__global__ void __launch_bounds__(THREADS, WQ_ROWS_MIN_BLOCKS) gemv_rows_kernel(const __grid_constant__ RowParamsT<CAP> P) {
   extern __shared__ __align__(16) uint32_t smem[];
   const int64_t share = (P.total_cost + gridDim.x - 1) / gridDim.x;
   const int64_t lo = share * blockIdx.x, hi = lo + share;
@@ -156,17 +174,22 @@ __global__ void __launch_bounds__(THREADS, WQ_ROWS_MIN_BLOCKS) gemv_rows_kernel(
     __syncthreads();
     for (int k8 = threadIdx.x; k8 < K / 8; k8 += THREADS) {
       const uint4 v = *reinterpret_cast<const uint4*>(M.x + 8 * k8);
-      if (XEXP) {
+      if (XM == 0) {
         reinterpret_cast<uint4*>(xs)[2 * k8] = make_uint4(v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16);
         reinterpret_cast<uint4*>(xs)[2 * k8 + 1] = make_uint4(v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16);
+      } else if (XM == 2) {  // (x0,x4) (x1,x5) (x2,x6) (x3,x7)
+        reinterpret_cast<uint4*>(xs)[k8] = make_uint4(prmt_u32(v.x, v.z, 0x5410), prmt_u32(v.x, v.z, 0x7632),
+                                                      prmt_u32(v.y, v.w, 0x5410), prmt_u32(v.y, v.w, 0x7632));
       } else {
         reinterpret_cast<uint4*>(xs)[k8] = v;
       }
     }
     __syncthreads();
 
-    for (int r0 = (int)r_lo; r0 < r_hi; r0 += THREADS) {
-      const int n = r0 + threadIdx.x;
+    // 32-row units dealt to the warps: a matrix boundary idles at most 31 lanes
+    const int nunits = (int)((r_hi - r_lo + 31) >> 5);
+    for (int u = threadIdx.x >> 5; u < nunits; u += THREADS / 32) {
+      const int n = (int)r_lo + 32 * u + (threadIdx.x & 31);
       if (n >= r_hi) continue;
       const uint8_t* crow = reinterpret_cast<const uint8_t*>(M.codes) + (size_t)n * (K * BITS / 8);
       const uint16_t* srow = M.scale + (size_t)n * G;
@@ -204,8 +227,8 @@ __global__ void __launch_bounds__(THREADS, WQ_ROWS_MIN_BLOCKS) gemv_rows_kernel(
           c[4 * ch + 3] = v.w;
         }
         float part;
-        if constexpr (BITS == 4) part = group_int4<XEXP>(c, xs, g * kGroup, m);
-        else part = group_int2<XEXP>(c, xs, g * kGroup, m);
+        if constexpr (BITS == 4) part = group_int4<XM>(c, xs, g * kGroup, m);
+        else part = group_int2<XM>(c, xs, g * kGroup, m);
         acc = fmaf(__half2float(__ushort_as_half((uint16_t)(m & 0xFFFFu))), part, acc);
       }
       cp_async_wait<0>();
@@ -239,14 +262,14 @@ bool rows_plan(RowParams& p, int bits, int count, const RowMatDesc* d, int* max_
   return kRowsStages * (kGroup * bits / 8) * kRowsThreads + (int64_t)mk * 4 <= kRowsMaxSmem;
 }
 
-template <int BITS, bool XEXP>
-static cudaError_t launch_t(const RowParams& p, int max_k, cudaStream_t stream) {
-  const int smem = kRowsStages * (kGroup * BITS / 8) * THREADS + max_k * (XEXP ? 4 : 2);
-  static int configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel<BITS, XEXP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsMaxSmem);
+template <int BITS, int XM, int CAP>
+static cudaError_t launch_cap(const RowParamsT<CAP>& p, int max_k, cudaStream_t stream) {
+  const int smem = kRowsStages * (kGroup * BITS / 8) * THREADS + max_k * (XM == 0 ? 4 : 2);
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel<BITS, XM, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsMaxSmem);
     if (e != cudaSuccess) return e;
-    configured = kRowsMaxSmem;
+    configured = true;
   }
   static int sms = 0;
   if (sms == 0) {
@@ -254,16 +277,26 @@ static cudaError_t launch_t(const RowParams& p, int max_k, cudaStream_t stream) 
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  gemv_rows_kernel<BITS, XEXP><<<WQ_ROWS_MIN_BLOCKS * sms, THREADS, smem, stream>>>(p);
+  gemv_rows_kernel<BITS, XM, CAP><<<WQ_ROWS_MIN_BLOCKS * sms, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
+template <int BITS, int XM>
+static cudaError_t launch_t(const RowParams& p, int max_k, cudaStream_t stream) {
+  if (p.count == 1) {
+    RowParamsT<1> p1;
+    p1.total_cost = p.total_cost;
+    p1.count = 1;
+    p1.m[0] = p.m[0];
+    return launch_cap<BITS, XM, 1>(p1, max_k, stream);
+  }
+  return launch_cap<BITS, XM, kRowsMaxMats>(p, max_k, stream);
+}
+
 cudaError_t launch_gemv_rows(const RowParams& p, int bits, int max_k, cudaStream_t stream) {
-#ifndef WQ_ROWS_PACKED_X
-  return bits == 4 ? launch_t<4, true>(p, max_k, stream) : launch_t<2, true>(p, max_k, stream);
-#else
-  return bits == 4 ? launch_t<4, false>(p, max_k, stream) : launch_t<2, false>(p, max_k, stream);
-#endif
+  // x layout in shared memory: int4 pairs x with the code pairs of a word (mode 2); int2
+  // codes pair (j, j + 8), so int2 uses the natural fp16-pair layout (mode 1)
+  return bits == 4 ? launch_t<4, WQ_ROWS_XMODE>(p, max_k, stream) : launch_t<2, (WQ_ROWS_XMODE == 0 ? 0 : 1)>(p, max_k, stream);
 }
 
 }  // namespace wq

@@ -24,11 +24,15 @@ struct RowMat {
   int N, K;
 };
 
-struct RowParams {
+// Passed by value as the kernel parameter; CAP is chosen per call (1 for a single matrix)
+// so that a launch copies no more parameter bytes than it uses.
+template <int CAP>
+struct RowParamsT {
   int64_t total_cost;
   int count;
-  RowMat m[kRowsMaxMats];
+  RowMat m[CAP];
 };
+using RowParams = RowParamsT<kRowsMaxMats>;
 
 struct RowMatDesc {
   const void* codes;
