@@ -227,7 +227,8 @@ def bench_rows(args, pk):
 
 
 def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 64, 512, 2048)):
-    """Batch sweep on the 0.5B set: one wq_gemm per matrix, the 169 calls in a CUDA graph."""
+    """Batch sweep on the 0.5B set: M tokens through all 169 matrices in one wq_linear_set
+    call per pass (tensor-core launches of up to 80 matrices for M >= 16)."""
     from bit_weight_quantized_unpack_b200 import wq
     wl = workloads.WORKLOADS[4]
     mats = workloads.workload_mats(4)
@@ -244,23 +245,19 @@ def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 64, 512, 2048)):
         X = [synth.activations(M, m.K, synth.sub_seed(wl["seed"], i, 1), device="cuda")
              for i, m in enumerate(mats)]
         Y = [torch.empty(M, m.N, dtype=torch.float16, device="cuda") for m in mats]
+        desc = wq.make_linear_set([(c, s, z, x, y, m.N, m.K, M)
+                                   for (c, s, z), m, x, y in zip(packed, mats, X, Y)])
 
-        def one_pass():
-            for (c, s, z), m, x, y in zip(packed, mats, X, Y):
-                wq.wq_gemm(x, M, c, s, z, "int4", m.N, m.K, y)
-        one_pass()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            one_pass()
+        def one_pass(i, desc=desc):
+            wq.wq_linear_set(desc, len(mats), "int4")
         steps = 20 if M >= 512 else 50
-        ms = time_steps(lambda i: g.replay(), steps if not args.quick else 5, 3, 1)
+        ms = time_steps(one_pass, steps if not args.quick else 5, 3, 1)
         flops = 2.0 * M * weights
         out[f"gemm_set_M{M}"] = {"ms": ms, "TFLOPS": flops / ms / 1e9,
                                  "frac_tensor": flops / ms / 1e9 / pk["bf16_tflops"],
                                  "weight_GBps": weights * INT4_BYTES_PER_WEIGHT / ms / 1e6,
-                                 "launches_per_pass": len(mats)}
-        del g, X, Y
+                                 "launches_per_pass": (len(mats) + 79) // 80 if M >= 16 else 1}
+        del X, Y
         torch.cuda.empty_cache()
     return out
 
@@ -315,7 +312,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(nbytes / ms / 1e6, 2),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(nbytes / ms / 1e6 / pk["hbm_gbs"], 4),
-                         "traffic": None, "kernel": "gemv_bulk_kernel<4>",
+                         "traffic": None, "kernel": "gemv_rows_kernel<4, 1, 256>",
                          "peak_source": pk["source"]},
             "e2e": {"value": round(nbytes * ws / ms_e2e / 1e6, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * K_tot, "d2h_bytes_per_step": 2 * N_tot},
@@ -325,7 +322,7 @@ def run_ours(args):
             "gemm_m512": ({"TFLOPS": round(rows["gemm_set_M512"]["TFLOPS"], 1),
                            "frac_of_tensor_peak": round(rows["gemm_set_M512"]["frac_tensor"], 4),
                            "peak_tflops": pk["bf16_tflops"],
-                           "workload": "qwen2.5-0.5b set, M=512, one wq_gemm per matrix in a CUDA graph"}
+                           "workload": "qwen2.5-0.5b set, M=512, one wq_linear_set call per pass"}
                           if "gemm_set_M512" in rows else None),
             "rows": rows,
         }
@@ -428,11 +425,20 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--quick", action="store_true", help="smaller rows / CPU sample")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
+    ap.add_argument("--case", default=None, choices=["gemm_set"],
+                    help="time one secondary case alone (for profiling): gemm_set = the "
+                         "0.5B set at --batch tokens through wq_linear_set")
+    ap.add_argument("--batch", type=int, default=512)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.case == "gemm_set":
+        torch.cuda.init()
+        args.quick = False
+        r = bench_batch_sweep(args, peaks(), Ms=(args.batch,))
+        print(json.dumps({"case": args.case, "batch": args.batch, **r}), flush=True)
     else:
         run_ours(args)
 

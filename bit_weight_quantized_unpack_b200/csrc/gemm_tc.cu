@@ -36,9 +36,18 @@ namespace {
 
 constexpr int BM = 128;       // weight rows per tile
 constexpr int BK = 64;        // k per stage: one 128-byte swizzle row of fp16
-constexpr int XSTAGES = 4;    // activation tiles [bn x 64] (read from L2)
-constexpr int CRING = 12;     // per-thread ring of code chunks: 11 k-blocks in flight
-constexpr int ASTAGES = 2;    // dequantised weight tiles (written by CUDA cores, read by MMA)
+#ifndef WQ_TC_XSTAGES
+#define WQ_TC_XSTAGES 4
+#endif
+#ifndef WQ_TC_ASTAGES
+#define WQ_TC_ASTAGES 2
+#endif
+#ifndef WQ_TC_CRING
+#define WQ_TC_CRING 12
+#endif
+constexpr int XSTAGES = WQ_TC_XSTAGES;  // activation tiles [bn x 64] (read from L2)
+constexpr int CRING = WQ_TC_CRING;      // per-thread ring of code chunks, CRING - 1 k-blocks in flight
+constexpr int ASTAGES = WQ_TC_ASTAGES;  // dequantised weight tiles (written by CUDA cores, read by MMA)
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB of dequantised fp16 weights
 constexpr int B_BYTES = kTcMaxBN * BK * 2;      // 32 KB of activations
 constexpr int CR_BYTES = BM * BK / 2;          // 4 KB of int4 codes per k-block
@@ -55,6 +64,7 @@ constexpr int THREADS = 512;                    // 16 warps
 constexpr int XPROD_WARP = 4, MMA_WARP = 5, DEQ_WARP0 = 8, DEQ_WARPS = 8;
 constexpr int TMEM_COLS = 2 * kTcMaxBN;         // two accumulator buffers
 static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled operands need 1 KB alignment");
+static_assert(SMEM_USED + 1024 <= 232448, "shared memory per block");
 
 __device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* gsrc) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");

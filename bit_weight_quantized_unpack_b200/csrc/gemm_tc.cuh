@@ -8,7 +8,8 @@
 namespace wq {
 
 constexpr int kTcMaxBN = 256;   // tokens per tile (MMA N), also the TMEM columns allocated
-constexpr int kTcMaxMats = 48;  // matrices per launch (tensor maps travel as kernel params)
+constexpr int kTcMaxMats = 80;  // matrices per launch: 80 x 384 B of tensor maps and fields fit
+                                // the 32 KB kernel parameter block
 constexpr int kTcMinM = 16;     // wq_gemm uses the tensor-core path from this M up (int4)
 
 // One matrix: tiles [tile_begin, tile_end) of the launch, tiles_m token tiles per

@@ -171,14 +171,14 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
     return cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
   }
   if (M == 1) {
-    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K};
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, 1};
     bool done = false;
     const int r = try_rows(fmt, 1, &d, (cudaStream_t)stream, &done);
     if (done) return r;
   }
   if (M == 1 && fmt != WQ_TERNARY && kUseBulkGemv) {
     static thread_local wq::BulkParams bp;
-    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K};
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, 1};
     if (plan_bulk(bp, fmt, 1, &d)) return cuda_status(wq::launch_gemv_bulk(bp, fmt == WQ_INT4 ? 4 : 2, (cudaStream_t)stream));
   }
   wq::SetParams p;
@@ -199,17 +199,20 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   if (!descs || count < 1 || count > WQ_LINEAR_SET_MAX) return WQ_ERR_ARG;
   if (fmt < WQ_INT4 || fmt > WQ_TERNARY) return WQ_ERR_ARG;
   static_assert(WQ_LINEAR_SET_MAX == wq::kSetMax, "set size");
-  wq::SetParams p;
+  static thread_local wq::SetParams p;
   p.count = count;
   int64_t total = 0;
+  const int64_t M = descs[0].M;
   for (int i = 0; i < count; ++i) {
     const wq_linear_desc& d = descs[i];
     int st = check_shape(fmt, d.N, d.K);
     if (st != WQ_OK) return st;
+    if (d.M < 1 || d.M > 2048) return WQ_ERR_SHAPE;
+    if (d.M != M) return WQ_ERR_ARG;
     if (!d.x || !d.y) return WQ_ERR_ARG;
     if ((st = check_weights(fmt, d.codes, d.scale, d.zero)) != WQ_OK) return st;
     if (!aligned(d.x, 16) || !aligned(d.y, 2)) return WQ_ERR_ALIGN;
-    const int64_t items = plan_mat(p.m[i], fmt, d.codes, d.scale, d.zero, d.x, d.y, d.N, d.K, 1);
+    const int64_t items = plan_mat(p.m[i], fmt, d.codes, d.scale, d.zero, d.x, d.y, d.N, d.K, d.M);
     p.m[i].item_begin = (int)total;
     total += items;
     if (total > INT_MAX) return WQ_ERR_SHAPE;
@@ -217,7 +220,36 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   }
   int st0 = check_device();
   if (st0 != WQ_OK) return st0;
-  {
+  if (fmt == WQ_INT4 && M >= wq::kTcMinM) {
+    // tensor-core GEMM: persistent launches of up to kTcMaxMats matrices each
+    static thread_local wq::TcParams tp;
+    // as few launches as the parameter block allows, with equal matrix counts
+    const int launches = (count + wq::kTcMaxMats - 1) / wq::kTcMaxMats;
+    for (int l = 0, i0 = 0; l < launches; ++l) {
+      const int n = (count - i0) / (launches - l);
+      int tiles = 0;
+      int64_t cost = 0;
+      for (int j = 0; j < n; ++j) {
+        const wq_linear_desc& d = descs[i0 + j];
+        wq::TcMat& t = tp.m[j];
+        if (!wq::tc_plan_mat(t, d.x, (int)M, d.codes, d.scale, d.zero, d.y, (int)d.N, (int)d.K, wq::tc_bn_for((int)M)))
+          return WQ_ERR_CUDA;
+        t.tile_begin = tiles;
+        t.cost_begin = cost;
+        tiles += t.tiles_n * t.tiles_m;
+        cost += (int64_t)t.tiles_n * t.tiles_m * t.tile_cost;
+        t.tile_end = tiles;
+      }
+      tp.count = n;
+      tp.total_tiles = tiles;
+      tp.total_cost = cost;
+      const int st = cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
+      if (st != WQ_OK) return st;
+      i0 += n;
+    }
+    return WQ_OK;
+  }
+  if (M == 1) {
     bool done = false;
     const int r = try_rows(fmt, count, descs, (cudaStream_t)stream, &done);
     if (done) return r;
@@ -234,7 +266,7 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   p.total_items = (int)total;
   int st = check_device();
   if (st != WQ_OK) return st;
-  return cuda_status(wq::launch_gemv_set(p, fmt, 1, (cudaStream_t)stream));
+  return cuda_status(wq::launch_gemv_set(p, fmt, (int)M, (cudaStream_t)stream));
 }
 
 const char* wq_status_str(int status) {

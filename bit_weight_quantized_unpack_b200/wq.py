@@ -30,7 +30,7 @@ _i64, _p, _i = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
 
 class wq_linear_desc(ctypes.Structure):
     _fields_ = [("codes", _p), ("scale", _p), ("zero", _p), ("x", _p), ("y", _p),
-                ("N", _i64), ("K", _i64)]
+                ("N", _i64), ("K", _i64), ("M", _i64)]
 
 
 _sig = {
@@ -107,10 +107,12 @@ def wq_gemm(X, M, codes, scale, zero, fmt, N, K, Y, stream=None) -> None:
 
 
 def make_linear_set(entries) -> ctypes.Array:
-    """Host descriptor array from (codes, scale, zero, x, y, N, K) tuples."""
+    """Host descriptor array from (codes, scale, zero, x, y, N, K[, M]) tuples (M = 1 if omitted)."""
     arr = (wq_linear_desc * len(entries))()
-    for i, (c, s, z, x, y, N, K) in enumerate(entries):
-        arr[i] = wq_linear_desc(_ptr(c), _ptr(s), _ptr(z), _ptr(x), _ptr(y), N, K)
+    for i, e in enumerate(entries):
+        c, s, z, x, y, N, K = e[:7]
+        M = e[7] if len(e) > 7 else 1
+        arr[i] = wq_linear_desc(_ptr(c), _ptr(s), _ptr(z), _ptr(x), _ptr(y), N, K, M)
     return arr
 
 

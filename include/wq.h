@@ -100,27 +100,30 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
             const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* Y,
             void* stream);
 
-/* One matrix of a linear set: y = x . w_hat^T with this matrix's own x and y. */
+/* One matrix of a linear set: Y = X . w_hat^T with this matrix's own X and Y. */
 typedef struct {
   const void* codes;
   const uint16_t* scale;
   const uint16_t* zero;   /* NULL for WQ_TERNARY */
-  const uint16_t* x;      /* fp16 [K] */
-  uint16_t* y;            /* fp16 [N] */
+  const uint16_t* x;      /* fp16 [M, K] row-major (M = 1: one vector) */
+  uint16_t* y;            /* fp16 [M, N] row-major */
   int64_t N;
   int64_t K;
+  int64_t M;              /* rows of x and y, 1 <= M <= 2048 */
 } wq_linear_desc;
 
 /* Largest count accepted by wq_linear_set. */
 #define WQ_LINEAR_SET_MAX 256
 
-/* Run `count` independent matrix-vector products of one format in ONE persistent kernel
- * launch. `descs` is a HOST array (read during the call, not kept); the pointers inside
- * are device pointers. Equivalent to count wq_gemv calls, without count launches: at
- * batch 1 a whole decoded token reads every weight once, and per-launch overhead
- * dominates small matrices (Whetstone README, "The baseline, and where the opportunity
- * actually is": dispatch and launch overhead, not bytes, set the baseline's speed).
- * 1 <= count <= WQ_LINEAR_SET_MAX; each entry obeys the wq_gemv requirements. */
+/* Run `count` independent products of one format as ONE persistent kernel launch per kind
+ * of kernel (matrix-vector for M = 1, tensor-core GEMM for int4 with M >= 16 -- split into
+ * launches of at most 80 matrices --, streaming skinny kernel otherwise). `descs` is a
+ * HOST array (read during the call, not kept); the pointers inside are device pointers.
+ * Equivalent to count wq_gemm calls, without count launches: at batch 1 a whole decoded
+ * token reads every weight once, and per-launch overhead dominates small matrices
+ * (Whetstone README, "The baseline, and where the opportunity actually is": dispatch and
+ * launch overhead, not bytes, set the baseline's speed). All entries must have the same
+ * M. 1 <= count <= WQ_LINEAR_SET_MAX; each entry obeys the wq_gemm requirements. */
 int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream);
 
 /* Static string naming a status code. */

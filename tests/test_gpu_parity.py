@@ -115,6 +115,42 @@ def test_linear_set_small_matches_gemv_and_oracle():
 
 
 @pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M", [2, 5, 16, 37, 300])
+def test_linear_set_batched_matches_gemm_and_oracle(fmt, M):
+    """A set of M-row products (tensor-core path for int4 at M >= 16, over more matrices
+    than one tensor-core launch takes) equals per-matrix wq_gemm and the oracle."""
+    base = [(896, 896), (128, 896), (333, 1152), (40, 4864), (513, 256), (256, 128)]
+    shapes = base * (15 if (fmt == "int4" and M == 16) else 1)  # 90 > 80 matrices per launch
+    ent, checks = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = synth.weights(N, K, 0.02, seed=300 + i)
+        X = synth.activations(M, K, seed=400 + i)
+        c, s, z = quantize_gpu(W.cuda(), fmt)
+        Xd = X.cuda()
+        Y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+        Ys = torch.empty(M, N, dtype=torch.float16, device="cuda")
+        wq().wq_gemm(Xd, M, c, s, z, fmt, N, K, Ys)
+        ent.append((c, s, z, Xd, Y, N, K, M))
+        ref = oracle_rows(W.numpy(), X.numpy(), fmt)[1:] if i < len(base) else None
+        checks.append((Y, Ys, ref, (N, K)))
+    wq().wq_linear_set(wq().make_linear_set(ent), len(ent), fmt)
+    torch.cuda.synchronize()
+    for Y, Ys, ref, shp in checks:
+        assert torch.equal(Y, Ys), (fmt, M, shp)
+        if ref is not None:
+            assert_within_tol(f16_np(Y), ref[0], ref[1], f"set {fmt} M={M} {shp}")
+
+
+def test_linear_set_rejects_mixed_m():
+    c, s, z = quantize_gpu(synth.weights(128, 128, 0.02, 1).cuda(), "int4")
+    x = torch.zeros(2, 128, dtype=torch.float16, device="cuda")
+    y = torch.zeros(2, 128, dtype=torch.float16, device="cuda")
+    arr = wq().make_linear_set([(c, s, z, x, y, 128, 128, 2), (c, s, z, x, y, 128, 128, 1)])
+    with pytest.raises(wq().WQError):
+        wq().wq_linear_set(arr, 2, "int4")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 17])
 def test_gemm_small(fmt, M):
     N, K = 300, 1024
@@ -219,3 +255,28 @@ def test_workload4_batch_sweep_sampled(M):
         _, y_ref, bound = oracle_rows(Wr, X[torch.as_tensor(mrows, device="cuda")].cpu().numpy(), "int4")
         got = f16_np(Y)[np.ix_(mrows, rows)]
         assert_within_tol(got, y_ref, bound, f"gemm M={M} {m.name}")
+
+
+def test_workload4_full_set_m512_sampled():
+    """The prefill-sized batch over the whole 0.5B set in one call, as the bench times it."""
+    wl = workloads.WORKLOADS[4]
+    M = 512
+    mats = workloads.workload_mats(1)
+    ent, keep = [], []
+    for i, m in enumerate(mats):
+        W = synth.weights(m.N, m.K, wl["sigma"], synth.sub_seed(wl["seed"], i, 0), device="cuda")
+        c, s, z = quantize_gpu(W, "int4")
+        X = synth.activations(M, m.K, synth.sub_seed(wl["seed"], i, 1), device="cuda")
+        Y = torch.empty(M, m.N, dtype=torch.float16, device="cuda")
+        rows = _sample_rows(m.N, 4, i)
+        Wr = W[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+        del W
+        ent.append((c, s, z, X, Y, m.N, m.K, M))
+        keep.append((m, rows, Wr))
+    wq().wq_linear_set(wq().make_linear_set(ent), len(ent), "int4")
+    torch.cuda.synchronize()
+    for i, ((c, s, z, X, Y, N, K, _), (m, rows, Wr)) in enumerate(zip(ent, keep)):
+        mrows = _sample_rows(M, 3, 1000 + i)
+        _, y_ref, bound = oracle_rows(Wr, X[torch.as_tensor(mrows, device="cuda")].cpu().numpy(), "int4")
+        got = f16_np(Y)[np.ix_(mrows, rows)]
+        assert_within_tol(got, y_ref, bound, f"set M=512 {m.name}")
