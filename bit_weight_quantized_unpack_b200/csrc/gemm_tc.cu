@@ -117,6 +117,10 @@ __device__ int first_tile_at(const TcParamsT<CAP>& P, int64_t target) {
   return P.total_tiles;
 }
 
+struct SzPair {
+  uint16_t s, z;  // fp16 bits of one group's scale and zero
+};
+
 struct TileInfo {
   int mi, n0, m0, bn, nkb;
 };
@@ -240,11 +244,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     // two threads per weight row: thread pairs (2r, 2r+1) take k 0..31 and 32..63 of it
     const int t = threadIdx.x - 32 * DEQ_WARP0;
     const int r = t >> 1, h = t & 1;
-    // scale | zero << 16 of groups g, g+1 (loaded ahead); the next tile's first two groups
-    // are fetched near the end of the current tile so a tile start never waits on them
-    auto load_sz = [&](const TcMat& M, int n, int g) -> uint32_t {
+    // scale and zero of groups g, g+1 (loaded ahead); the next tile's first two groups
+    // are fetched near the end of the current tile so a tile start never waits on them.
+    // The two halves stay in separate registers until they are used: combining them at load
+    // time would stall the warp for the whole load latency.
+    auto load_sz = [&](const TcMat& M, int n, int g) -> SzPair {
       const int G = M.K / kGroup;
-      return (uint32_t)ld_u16(M.scale + (size_t)n * G + g) | ((uint32_t)ld_u16(M.zero + (size_t)n * G + g) << 16);
+      return {ld_u16(M.scale + (size_t)n * G + g), ld_u16(M.zero + (size_t)n * G + g)};
     };
     // Codes are not copied by TMA: a slow DRAM copy would hold up the activation copies
     // queued behind it. Each thread streams its own 16-byte chunk of every k-block of its
@@ -270,40 +276,39 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     };
     for (int i = 0; i < CRING - 1; ++i) fetch_next();
     int cseq = 0;
-    uint32_t pre0 = 0, pre1 = 0;
+    SzPair pre0{0, 0}, pre1{0, 0};
     int mi_pre = 0;
     if (t_lo < t_hi) {
       const TileInfo t0 = tile_info(P, t_lo, mi_pre);
       const TcMat& M0 = P.m[t0.mi];
       const int n = min(t0.n0 + r, M0.N - 1);
       pre0 = load_sz(M0, n, 0);
-      pre1 = M0.K > kGroup ? load_sz(M0, n, 1) : 0u;
+      if (M0.K > kGroup) pre1 = load_sz(M0, n, 1);
     }
     for (int tile = t_lo; tile < t_hi && !timed_out; ++tile) {
       const TileInfo ti = tile_info(P, tile, mi);
       const TcMat& M = P.m[ti.mi];
       const int n = min(ti.n0 + r, M.N - 1);  // rows past N are computed but never stored
       const int G = M.K / kGroup;
-      uint32_t sz0 = pre0, sz1 = pre1, sz2 = 0;
+      SzPair sz0 = pre0, sz1 = pre1;
       uint32_t c1024z = 0, s2 = 0;
       const int kb_pre = ti.nkb > 4 ? ti.nkb - 4 : 0;
       for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
         const int a = it % ASTAGES;
         if ((kb & 1) == 0) {
           const int g = kb >> 1;
-          if (g + 2 < G) sz2 = load_sz(M, n, g + 2);
-          const __half z = __ushort_as_half((uint16_t)(sz0 >> 16));
+          const __half z = __ushort_as_half(sz0.z);
           c1024z = pack_h2(__hadd(z, __float2half(1024.f)));
-          s2 = (sz0 & 0xFFFFu) | (sz0 << 16);
+          s2 = (uint32_t)sz0.s | ((uint32_t)sz0.s << 16);
           sz0 = sz1;
-          sz1 = sz2;
+          if (g + 2 < G) sz1 = load_sz(M, n, g + 2);
         }
         if (kb == kb_pre && tile + 1 < t_hi) {
           const TileInfo tn = tile_info(P, tile + 1, mi_pre);
           const TcMat& Mn = P.m[tn.mi];
           const int nn = min(tn.n0 + r, Mn.N - 1);
           pre0 = load_sz(Mn, nn, 0);
-          pre1 = Mn.K > kGroup ? load_sz(Mn, nn, 1) : 0u;
+          if (Mn.K > kGroup) pre1 = load_sz(Mn, nn, 1);
         }
         fetch_next();
         cp_async_wait_ring();  // this k-block's chunk (issued CRING - 1 fetches ago) has landed

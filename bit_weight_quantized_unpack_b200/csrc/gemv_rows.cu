@@ -26,11 +26,6 @@ namespace {
 
 constexpr int THREADS = kRowsThreads;
 
-// Metadata of one group: scale | zero << 16 (fp16 bits), through L1 (a row's metadata
-// shares one sector, so the following groups hit).
-__device__ __forceinline__ uint32_t ld_meta(const uint16_t* s, const uint16_t* z) {
-  return (uint32_t)ld_u16(s) | ((uint32_t)ld_u16(z) << 16);
-}
 
 // x value k of the staged activation vector as an f16 operand (low half of a word).
 template <int XM>
@@ -46,8 +41,8 @@ __device__ __forceinline__ uint16_t xval(const uint32_t* xs, int k) {
 // natural order; 2 = fp16 pairs (x_j, x_j+4) of each group of eight, matching the code
 // pairs of one word of codes, so both operands of every multiply sit in the same half.
 template <int XM>
-__device__ __forceinline__ float group_int4(const uint32_t (&c)[16], const uint32_t* xs, int k0, uint32_t sz) {
-  const __half z = __ushort_as_half((uint16_t)(sz >> 16));
+__device__ __forceinline__ float group_int4(const uint32_t (&c)[16], const uint32_t* xs, int k0, uint16_t zbits) {
+  const __half z = __ushort_as_half(zbits);
   const uint32_t c1 = pack_h2(__hadd(z, __float2half(1024.f)));
   const uint32_t c16 = pack_h2(__hfma(z, __float2half(16.f), __float2half(1024.f)));
   float a[2] = {0.f, 0.f}, b[2] = {0.f, 0.f};
@@ -97,8 +92,8 @@ __device__ __forceinline__ float group_int4(const uint32_t (&c)[16], const uint3
 
 // One int2 group (128 weights = 8 words in one sector).
 template <int XM>
-__device__ __forceinline__ float group_int2(const uint32_t (&c)[8], const uint32_t* xs, int k0, uint32_t sz) {
-  const __half z = __ushort_as_half((uint16_t)(sz >> 16));
+__device__ __forceinline__ float group_int2(const uint32_t (&c)[8], const uint32_t* xs, int k0, uint16_t zbits) {
+  const __half z = __ushort_as_half(zbits);
   constexpr uint32_t kMask[4] = {0x00030003u, 0x000C000Cu, 0x00300030u, 0x00C000C0u};
   uint32_t cz[4];
 #pragma unroll
@@ -203,7 +198,9 @@ __global__ void __launch_bounds__(THREADS, WQ_ROWS_MIN_BLOCKS) gemv_rows_kernel(
         }
         cp_async_commit();
       }
-      uint32_t m_next = ld_meta(srow, zrow);
+      // scale and zero of the next group, in separate registers until used (combining them
+      // right after the loads would stall the lane for the load latency)
+      uint16_t s_next = ld_u16(srow), z_next = ld_u16(zrow);
       float acc = 0.f;
       for (int g = 0; g < G; ++g) {
         // keep S-1 groups in flight: issue group g + S - 1, then wait for group g
@@ -214,8 +211,11 @@ __global__ void __launch_bounds__(THREADS, WQ_ROWS_MIN_BLOCKS) gemv_rows_kernel(
             cp_async16(ring_chunk<BITS>(ring, gi % S, ch), crow + (size_t)gi * GB + 16 * ch);
         }
         cp_async_commit();
-        const uint32_t m = m_next;
-        if (g + 1 < G) m_next = ld_meta(srow + g + 1, zrow + g + 1);
+        const uint16_t sc = s_next, zc = z_next;
+        if (g + 1 < G) {
+          s_next = ld_u16(srow + g + 1);
+          z_next = ld_u16(zrow + g + 1);
+        }
         cp_async_wait<S - 1>();
         uint32_t c[GB / 4];
 #pragma unroll
@@ -227,9 +227,9 @@ __global__ void __launch_bounds__(THREADS, WQ_ROWS_MIN_BLOCKS) gemv_rows_kernel(
           c[4 * ch + 3] = v.w;
         }
         float part;
-        if constexpr (BITS == 4) part = group_int4<XM>(c, xs, g * kGroup, m);
-        else part = group_int2<XM>(c, xs, g * kGroup, m);
-        acc = fmaf(__half2float(__ushort_as_half((uint16_t)(m & 0xFFFFu))), part, acc);
+        if constexpr (BITS == 4) part = group_int4<XM>(c, xs, g * kGroup, zc);
+        else part = group_int2<XM>(c, xs, g * kGroup, zc);
+        acc = fmaf(__half2float(__ushort_as_half(sc)), part, acc);
       }
       cp_async_wait<0>();
       M.y[n] = __half_as_ushort(__float2half_rn(acc));
