@@ -37,34 +37,35 @@ namespace {
 constexpr int BM = 128;       // weight rows per tile
 constexpr int BK = 64;        // k per stage: one 128-byte swizzle row of fp16
 #ifndef WQ_TC_XSTAGES
-#define WQ_TC_XSTAGES 4
+#define WQ_TC_XSTAGES 3
 #endif
 #ifndef WQ_TC_ASTAGES
-#define WQ_TC_ASTAGES 2
+#define WQ_TC_ASTAGES 4
 #endif
 #ifndef WQ_TC_CRING
-#define WQ_TC_CRING 12
+#define WQ_TC_CRING 6
 #endif
 constexpr int XSTAGES = WQ_TC_XSTAGES;  // activation tiles [bn x 64] (read from L2)
-constexpr int CRING = WQ_TC_CRING;      // per-thread ring of code chunks, CRING - 1 k-blocks in flight
+constexpr int CRING = WQ_TC_CRING;      // codes ring slots: CRING - 1 of a team's k-blocks in flight
 constexpr int ASTAGES = WQ_TC_ASTAGES;  // dequantised weight tiles (written by CUDA cores, read by MMA)
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB of dequantised fp16 weights
 constexpr int B_BYTES = kTcMaxBN * BK * 2;      // 32 KB of activations
-constexpr int CR_BYTES = BM * BK / 2;          // 4 KB of int4 codes per k-block
+constexpr int CSLOT_BYTES = 2 * BM * BK / 2;   // one ring slot: 32 B of codes for each of 256 threads
 constexpr int OFF_A = 0;
 constexpr int OFF_X = OFF_A + ASTAGES * A_BYTES;
 constexpr int OFF_C = OFF_X + XSTAGES * B_BYTES;
 constexpr int EPI_BYTES = 32 * 32 * 2;          // one warp's 32 x 32 fp16 output block
-constexpr int OFF_E = OFF_C + CRING * CR_BYTES;  // [4 warps][2 buffers] staged output blocks
+constexpr int OFF_E = OFF_C + CRING * CSLOT_BYTES;  // [4 warps][2 buffers] staged output blocks
 constexpr int OFF_BAR = OFF_E + 4 * 2 * EPI_BYTES;
 constexpr int NUM_BARS = 2 * XSTAGES + 2 * ASTAGES + 4;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
 constexpr int THREADS = 512;                    // 16 warps
-constexpr int XPROD_WARP = 4, MMA_WARP = 5, DEQ_WARP0 = 8, DEQ_WARPS = 8;
+constexpr int XPROD_WARP = 4, MMA_WARP = 5, DEQ_WARP0 = 8, DEQ_WARPS = 8, TEAM_WARPS = 4;
 constexpr int TMEM_COLS = 2 * kTcMaxBN;         // two accumulator buffers
 static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled operands need 1 KB alignment");
 static_assert(SMEM_USED + 1024 <= 232448, "shared memory per block");
+static_assert(DEQ_WARPS == 2 * TEAM_WARPS && TEAM_WARPS * 32 == BM, "two teams, one row per thread");
 
 __device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* gsrc) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc) : "memory");
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
       tc::mbar_init(bar_xempty + 8 * i, 1);
     }
     for (int i = 0; i < ASTAGES; ++i) {
-      tc::mbar_init(bar_aready + 8 * i, DEQ_WARPS);
+      tc::mbar_init(bar_aready + 8 * i, TEAM_WARPS);
       tc::mbar_init(bar_aempty + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -241,91 +242,100 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
       }
     }
   } else if (warp >= DEQ_WARP0) {
-    // two threads per weight row: thread pairs (2r, 2r+1) take k 0..31 and 32..63 of it
-    const int t = threadIdx.x - 32 * DEQ_WARP0;
-    const int r = t >> 1, h = t & 1;
-    // scale and zero of groups g, g+1 (loaded ahead); the next tile's first two groups
-    // are fetched near the end of the current tile so a tile start never waits on them.
-    // The two halves stay in separate registers until they are used: combining them at load
-    // time would stall the warp for the whole load latency.
+    // Two teams of four warps; team e dequantises the k-blocks with it % 2 == e, so each
+    // warp has two k-block periods for one k-block's work and its fixed costs (waits,
+    // fence, arrive) are paid once per 64 k of a row. Thread r of a team owns weight row r.
+    const int t = threadIdx.x - 32 * DEQ_WARP0;   // 0 .. 255 (slot of the codes ring)
+    const int team = t >> 7, r = t & 127;
+    // scale and zero of the team's next two k-blocks (one k-block per 128-k group and team),
+    // in separate registers until used: combining them at load time would stall the warp
+    // for the whole load latency.
     auto load_sz = [&](const TcMat& M, int n, int g) -> SzPair {
       const int G = M.K / kGroup;
       return {ld_u16(M.scale + (size_t)n * G + g), ld_u16(M.zero + (size_t)n * G + g)};
     };
+    // A cursor over this CTA's (tile, k-block) sequence restricted to one team's k-blocks.
+    struct Cursor {
+      int tile, kb, mi;
+      TileInfo ti;
+    };
+    auto cursor_start = [&](Cursor& c) {
+      c.tile = t_lo;
+      c.kb = team;
+      c.mi = 0;
+      if (c.tile < t_hi) c.ti = tile_info(P, c.tile, c.mi);
+    };
+    auto cursor_next = [&](Cursor& c) {
+      c.kb += 2;
+      if (c.kb >= c.ti.nkb) {
+        c.kb = team;
+        if (++c.tile < t_hi) c.ti = tile_info(P, c.tile, c.mi);
+      }
+    };
     // Codes are not copied by TMA: a slow DRAM copy would hold up the activation copies
-    // queued behind it. Each thread streams its own 16-byte chunk of every k-block of its
-    // row with cp.async into its slot of a CRING-deep ring ([slot][thread] x 16 bytes),
-    // CRING - 1 k-blocks ahead, across tile boundaries.
-    const uint32_t cring = sbase + OFF_C + 16u * (uint32_t)t;
-    int f_tile = t_lo, f_kb = 0, f_mi = 0, fseq = 0;
-    TileInfo f_ti{};
-    if (f_tile < t_hi) f_ti = tile_info(P, f_tile, f_mi);
+    // queued behind it. Each thread streams the 32 bytes of its row in each of the team's
+    // k-blocks with two cp.async copies into its slot of a CRING-deep ring
+    // ([slot][16-byte half][thread]), CRING - 1 of the team's k-blocks ahead, across tiles.
+    Cursor fc;
+    cursor_start(fc);
+    int fseq = 0;
     auto fetch_next = [&]() {
-      if (f_tile < t_hi) {
-        const TcMat& Mf = P.m[f_ti.mi];
-        const int nf = min(f_ti.n0 + r, Mf.N - 1);
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(Mf.codes) + (size_t)nf * (Mf.K / 2) + f_kb * (BK / 2) + h * 16;
-        cp_async16(cring + (uint32_t)(fseq % CRING) * (CR_BYTES), src);
-        if (++f_kb == f_ti.nkb) {
-          f_kb = 0;
-          if (++f_tile < t_hi) f_ti = tile_info(P, f_tile, f_mi);
-        }
+      if (fc.tile < t_hi) {
+        const TcMat& Mf = P.m[fc.ti.mi];
+        const int nf = min(fc.ti.n0 + r, Mf.N - 1);
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(Mf.codes) + (size_t)nf * (Mf.K / 2) + fc.kb * (BK / 2);
+        const uint32_t dst = sbase + OFF_C + (uint32_t)(fseq % CRING) * CSLOT_BYTES + 16u * (uint32_t)t;
+        cp_async16(dst, src);
+        cp_async16(dst + CSLOT_BYTES / 2, src + 16);
+        cursor_next(fc);
       }
       cp_async_commit();
       ++fseq;
     };
     for (int i = 0; i < CRING - 1; ++i) fetch_next();
+    // scale / zero prefetch cursor, two of the team's k-blocks ahead
+    Cursor sc;
+    cursor_start(sc);
+    SzPair sz0{0, 0}, sz1{0, 0};
+    auto sz_fetch = [&]() -> SzPair {
+      SzPair v{0, 0};
+      if (sc.tile < t_hi) {
+        const TcMat& Ms = P.m[sc.ti.mi];
+        v = load_sz(Ms, min(sc.ti.n0 + r, Ms.N - 1), sc.kb >> 1);
+        cursor_next(sc);
+      }
+      return v;
+    };
+    sz0 = sz_fetch();
+    sz1 = sz_fetch();
     int cseq = 0;
-    SzPair pre0{0, 0}, pre1{0, 0};
-    int mi_pre = 0;
-    if (t_lo < t_hi) {
-      const TileInfo t0 = tile_info(P, t_lo, mi_pre);
-      const TcMat& M0 = P.m[t0.mi];
-      const int n = min(t0.n0 + r, M0.N - 1);
-      pre0 = load_sz(M0, n, 0);
-      if (M0.K > kGroup) pre1 = load_sz(M0, n, 1);
-    }
     for (int tile = t_lo; tile < t_hi && !timed_out; ++tile) {
       const TileInfo ti = tile_info(P, tile, mi);
-      const TcMat& M = P.m[ti.mi];
-      const int n = min(ti.n0 + r, M.N - 1);  // rows past N are computed but never stored
-      const int G = M.K / kGroup;
-      SzPair sz0 = pre0, sz1 = pre1;
-      uint32_t c1024z = 0, s2 = 0;
-      const int kb_pre = ti.nkb > 4 ? ti.nkb - 4 : 0;
-      for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-        const int a = it % ASTAGES;
-        if ((kb & 1) == 0) {
-          const int g = kb >> 1;
-          const __half z = __ushort_as_half(sz0.z);
-          c1024z = pack_h2(__hadd(z, __float2half(1024.f)));
-          s2 = (uint32_t)sz0.s | ((uint32_t)sz0.s << 16);
-          sz0 = sz1;
-          if (g + 2 < G) sz1 = load_sz(M, n, g + 2);
-        }
-        if (kb == kb_pre && tile + 1 < t_hi) {
-          const TileInfo tn = tile_info(P, tile + 1, mi_pre);
-          const TcMat& Mn = P.m[tn.mi];
-          const int nn = min(tn.n0 + r, Mn.N - 1);
-          pre0 = load_sz(Mn, nn, 0);
-          if (Mn.K > kGroup) pre1 = load_sz(Mn, nn, 1);
-        }
+      for (int kb = team; kb < ti.nkb; kb += 2) {
+        const int itk = it + kb;               // sequence number of this k-block
+        const int a = itk % ASTAGES;
+        const __half z = __ushort_as_half(sz0.z);
+        const uint32_t c1024z = pack_h2(__hadd(z, __float2half(1024.f)));
+        const uint32_t s2 = (uint32_t)sz0.s | ((uint32_t)sz0.s << 16);
+        sz0 = sz1;
+        sz1 = sz_fetch();
         fetch_next();
-        cp_async_wait_ring();  // this k-block's chunk (issued CRING - 1 fetches ago) has landed
-        if (!tc::mbar_wait(bar_aempty + 8 * a, ((it / ASTAGES) & 1) ^ 1)) { timed_out = true; break; }
-        const uint4 cw = *reinterpret_cast<const uint4*>(smem + OFF_C + (cseq % CRING) * CR_BYTES + 16 * t);
+        cp_async_wait_ring();  // this k-block's codes (issued CRING - 1 fetches ago) have landed
+        if (!tc::mbar_wait(bar_aempty + 8 * a, ((itk / ASTAGES) & 1) ^ 1)) { timed_out = true; break; }
+        const uint8_t* cslot = smem + OFF_C + (cseq % CRING) * CSLOT_BYTES + 16 * t;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(cslot);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(cslot + CSLOT_BYTES / 2);
         ++cseq;
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         uint8_t* arow = smem + OFF_A + a * A_BYTES + r * 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = 4 * h + i;  // logical 16-byte chunk (8 fp16) within the 128-byte row
-          *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = dequant8(words[i], c1024z, s2);
-        }
+        for (int j = 0; j < 8; ++j)  // logical 16-byte chunk (8 fp16) j of the 128-byte row
+          *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) = dequant8(words[j], c1024z, s2);
         tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(bar_aready + 8 * a);
       }
+      it += ti.nkb;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp < 4) {
