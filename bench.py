@@ -312,7 +312,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(nbytes / ms / 1e6, 2),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(nbytes / ms / 1e6 / pk["hbm_gbs"], 4),
-                         "traffic": None, "kernel": "gemv_rows_kernel<4, 1, 256>",
+                         "traffic": None, "kernel": "gemv_stream_kernel<4, 256>",
                          "peak_source": pk["source"]},
             "e2e": {"value": round(nbytes * ws / ms_e2e / 1e6, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * K_tot, "d2h_bytes_per_step": 2 * N_tot},

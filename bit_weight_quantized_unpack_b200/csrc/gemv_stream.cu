@@ -1,0 +1,537 @@
+// Matrix-vector product against packed int4 / int2 weights, streamed as contiguous bytes.
+//
+// Whetstone README, "The one fact that shapes everything": at batch 1 every weight is read
+// once for one multiply-add, so the product runs at the speed the packed codes stream from
+// HBM. On B200 that speed needs long contiguous reads: rows are contiguous in memory, so
+// each warp owns a contiguous range of whole rows and moves it into shared memory with
+// cp.async.bulk copies (2 KB of codes plus their scales and zeros per copy, a ring of a few
+// copies in flight per warp, completion on mbarriers).
+//
+// The staged bytes are a stream of cells, one cell = one row's 128-weight group (64 bytes
+// of int4 codes, 32 of int2). Lane j takes cell j of each step of 32 cells. Its 16-byte
+// chunks are read in an order rotated by the cell's group index, so that the eight lanes of
+// a shared-memory phase hit eight different bank groups and lanes holding the same group
+// index read the same activations (a broadcast); the activation vector is staged with 17
+// units of 16 bytes per group (one spare) for the same reason.
+//
+// Dequantisation is one AND per pair of codes: the masked bits of a binary16 lane are the
+// subnormal number q * 2^-24 (16 q * 2^-24 for the high nibble of a byte, which stays below
+// the subnormal limit of 1024 * 2^-24); one packed binary16 subtract of z * 2^-24 (the
+// integer zero point as bits) gives (q - z) * 2^-24 exactly; each product with an fp16
+// activation is exact in binary32 (mixed-precision FMA); the 2^24 returns, exactly, with
+// the group scale. Only binary32 adds, the multiply by the scale and the final fp16 store
+// round, and q = z gives an exact zero. The cells of one row sit in
+// consecutive lanes (and steps): a segmented shuffle scan per step sums them, a carry
+// holds the part of a row that continues into the next step, and the lane holding a row's
+// last group writes y.
+//
+// The activation vector of the matrix being processed is staged once per CTA; two buffers
+// let the next matrix's vector load while the current one is in use.
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv_stream.cuh"
+#include "tc_ptx.cuh"
+
+namespace wq {
+
+namespace {
+
+constexpr int W = kStreamWarps;
+constexpr int T = 32 * W;
+constexpr int SLOT_CODES = kStreamSlotCodes;
+constexpr int XU = 17;  // staged activation units (16 bytes) per 128-weight group
+
+template <int BITS>
+struct Fmt {
+  static constexpr int CB = 128 * BITS / 8;    // codes bytes per cell (one group): 64 / 32
+  static constexpr int CH = CB / 16;           // 16-byte chunks per cell: 4 / 2
+  static constexpr int UPC = 16 / CH;          // activation units per chunk: 4 / 8
+  static constexpr int SPS = SLOT_CODES / (32 * CB);  // steps of 32 cells per ring slot: 2 / 4
+  static constexpr int GPSL = SLOT_CODES / CB;        // groups per ring slot: 64 / 128
+  static constexpr int META = 2 * GPSL;               // bytes of scales (and of zeros) per slot
+  static constexpr int SLOT = SLOT_CODES + 2 * META;
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint16_t lds16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+
+// Dot products of one 16-byte chunk of codes with its activations (shared-memory address
+// xa), accumulated in binary32 with the factor 2^-24 described above.
+// int4: 32 codes; z1 / z16 hold z and 16 z as binary16 bit patterns in both lanes; the A
+// accumulators take codes at bits 0-3 of a byte, the B ones (16x) bits 4-7.
+__device__ __forceinline__ void chunk_int4(const uint4 c, uint32_t xa, uint32_t z1, uint32_t z16, float& a0,
+                                           float& a1, float& b0, float& b1) {
+  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t v = cw[i], v8 = v >> 8;
+    const uint32_t d0 = hsub2_u32(v & 0x000F000Fu, z1);    // q0, q4
+    const uint32_t d1 = hsub2_u32(v & 0x00F000F0u, z16);   // 16 q1, 16 q5
+    const uint32_t d2 = hsub2_u32(v8 & 0x000F000Fu, z1);   // q2, q6
+    const uint32_t d3 = hsub2_u32(v8 & 0x00F000F0u, z16);  // 16 q3, 16 q7
+    const uint4 xw = lds128(xa + 16 * i);  // (x0, x1) (x2, x3) (x4, x5) (x6, x7)
+    float& A = (i & 1) ? a1 : a0;
+    float& B = (i & 1) ? b1 : b0;
+    A = fma_f16f16_f32(lo16(d0), lo16(xw.x), A);
+    A = fma_f16f16_f32(hi16(d0), lo16(xw.z), A);
+    A = fma_f16f16_f32(lo16(d2), lo16(xw.y), A);
+    A = fma_f16f16_f32(hi16(d2), lo16(xw.w), A);
+    B = fma_f16f16_f32(lo16(d1), hi16(xw.x), B);
+    B = fma_f16f16_f32(hi16(d1), hi16(xw.z), B);
+    B = fma_f16f16_f32(lo16(d3), hi16(xw.y), B);
+    B = fma_f16f16_f32(hi16(d3), hi16(xw.w), B);
+  }
+}
+
+// int2: 64 codes (four words of 16); zm[m] holds 4^m z as binary16 bits in both lanes; the
+// lanes of d are codes j and j + 8 of a word, scaled by 4^(j mod 4), accumulated in a[j mod 4].
+__device__ __forceinline__ void chunk_int2(const uint4 c, uint32_t xa, const uint32_t (&zm)[4], float (&a)[4]) {
+  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t v = cw[i], v8 = v >> 8;
+    const uint4 xl = lds128(xa + 32 * i), xh = lds128(xa + 32 * i + 16);  // x0 .. x7, x8 .. x15
+    const uint32_t xlw[4] = {xl.x, xl.y, xl.z, xl.w}, xhw[4] = {xh.x, xh.y, xh.z, xh.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t d = hsub2_u32((j < 4 ? v : v8) & (0x00030003u << (2 * (j & 3))), zm[j & 3]);
+      const uint16_t xj = (j & 1) ? hi16(xlw[j >> 1]) : lo16(xlw[j >> 1]);
+      const uint16_t xj8 = (j & 1) ? hi16(xhw[j >> 1]) : lo16(xhw[j >> 1]);
+      a[j & 3] = fma_f16f16_f32(lo16(d), xj, a[j & 3]);
+      a[j & 3] = fma_f16f16_f32(hi16(d), xj8, a[j & 3]);
+    }
+  }
+}
+
+// 2^-24 * sum_k x_k (q_k - z) over one cell at shared address `cell`; xg: shared address of
+// the group's activation units; oc[c] / ox[c]: offsets of the cell's c-th chunk in this
+// lane's rotated order and of that chunk's first activation unit.
+template <int BITS>
+__device__ __forceinline__ float cell_dot(uint32_t cell, uint32_t xg, const int (&oc)[Fmt<BITS>::CH],
+                                          const int (&ox)[Fmt<BITS>::CH], uint16_t zbits) {
+  using F = Fmt<BITS>;
+  const uint32_t zi = (uint32_t)__half2int_rn(__ushort_as_half(zbits));  // integer zero point
+  if constexpr (BITS == 4) {
+    const uint32_t z1 = zi * 0x00010001u, z16 = zi * 0x00100010u;
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < F::CH; ++c) chunk_int4(lds128(cell + oc[c]), xg + ox[c], z1, z16, a0, a1, b0, b1);
+    return fmaf(b0 + b1, 0.0625f, a0 + a1);
+  } else {
+    uint32_t zm[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) zm[m] = (zi << (2 * m)) * 0x00010001u;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < F::CH; ++c) chunk_int2(lds128(cell + oc[c]), xg + ox[c], zm, a);
+    return fmaf(a[3], 0.015625f, fmaf(a[2], 0.0625f, fmaf(a[1], 0.25f, a[0])));
+  }
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Units (RA rows each) of M whose first byte of cost lies in [lo, hi): [b0, b1).
+__device__ __forceinline__ void cta_units(const StreamMat& M, int64_t lo, int64_t hi, int& b0, int& b1) {
+  const int64_t bc = M.unit_cost;
+  const int64_t a = lo <= M.cost_begin ? 0 : (lo - M.cost_begin + bc - 1) / bc;
+  const int64_t b = hi <= M.cost_begin ? 0 : (hi - M.cost_begin + bc - 1) / bc;
+  b0 = (int)(a < M.nunit ? a : M.nunit);
+  b1 = (int)(b < M.nunit ? b : M.nunit);
+}
+
+// One warp's share of a matrix: whole units [wb0, wb1) of the CTA's range, as rows.
+struct Seg {
+  const uint8_t* codes;
+  const uint16_t* s;
+  const uint16_t* z;
+  int rows;
+  int row0;
+  int64_t bytes;   // codes bytes
+  int64_t groups;  // rows * K / 128
+};
+
+template <int BITS>
+__device__ __forceinline__ Seg warp_seg(const StreamMat& M, int b0, int b1, int w) {
+  const int wb0 = b0 + (int)((int64_t)(b1 - b0) * w / W);
+  const int wb1 = b0 + (int)((int64_t)(b1 - b0) * (w + 1) / W);
+  const int64_t r0 = (int64_t)wb0 * M.RA;
+  const int64_t r1 = (int64_t)wb1 * M.RA < M.N ? (int64_t)wb1 * M.RA : M.N;
+  const int64_t rb = (int64_t)M.K * BITS / 8;
+  const int G = M.K / kGroup;
+  Seg s;
+  s.rows = r1 > r0 ? (int)(r1 - r0) : 0;
+  s.row0 = (int)r0;
+  s.codes = reinterpret_cast<const uint8_t*>(M.codes) + r0 * rb;
+  s.s = M.scale + r0 * G;
+  s.z = M.zero + r0 * G;
+  s.bytes = (int64_t)s.rows * rb;
+  s.groups = (int64_t)s.rows * G;
+  return s;
+}
+
+// Copy state of one warp's producer (lane 0): what remains of the current segment.
+struct Prod {
+  const uint8_t* c;
+  const uint16_t* s;
+  const uint16_t* z;
+  int cleft;  // codes bytes not yet issued
+  int gleft;  // groups not yet issued
+  int pm;     // matrix of the segment
+};
+
+// Consume one warp segment from the ring: cells in order, lane j taking cell j of each step.
+template <int BITS, class Issue>
+__device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint8_t* ring,
+                                        uint64_t* bars, int slots, int& cslot, uint32_t& cphase, int& consumed,
+                                        bool& dead, Issue& issue, int lane) {
+  using F = Fmt<BITS>;
+  const int G = M.K / kGroup;
+  const int ncells = (int)seg.groups;
+  const int nsteps = (ncells + 31) / 32;
+  uint16_t* y = M.y + seg.row0;
+  // the matrix's last partial 16-byte unit of scales / zeros, if this segment ends there:
+  // loaded now, stored into its ring slot before that slot is read
+  const int rem = ncells & 7;
+  uint16_t rs = 0, rz = 0;
+  if (rem) {
+    const int gb = ncells - rem;
+    if (lane < rem) rs = ld_u16(seg.s + gb + lane);
+    if (lane >= 8 && lane < 8 + rem) rz = ld_u16(seg.z + gb + lane - 8);
+  }
+  // group gp of row `row` of the segment: this lane's cell
+  int gp = lane % G, row = lane / G;
+  const uint32_t gmul = ((1u << 20) + G - 1) / G;  // floor(n / G) = (n * gmul) >> 20 for n < G + 32, G < 32
+  float carry = 0.f;  // part of the row that continues from the previous step
+  for (int st = 0; st < nsteps; ++st) {
+    const int ss = st % F::SPS;
+    uint8_t* slot = ring + (size_t)cslot * F::SLOT;
+    if (ss == 0) {
+      if (!dead) {
+        const bool ok = tc::mbar_wait(tc::smem_u32(bars + cslot), cphase);
+        if (!__all_sync(0xffffffffu, ok)) dead = true;
+      }
+      if (rem && (st + F::SPS >= nsteps)) {  // the segment's last slot
+        const int gl = ncells - rem - (st / F::SPS) * F::GPSL;
+        uint16_t* sm = reinterpret_cast<uint16_t*>(slot + SLOT_CODES);
+        if (lane < rem) sm[gl + lane] = rs;
+        if (lane >= 8 && lane < 8 + rem) sm[F::META / 2 + gl + lane - 8] = rz;
+        tc::fence_proxy_async_smem();  // the slot is refilled by bulk copies later
+        __syncwarp();
+      }
+    }
+    const bool valid = st * 32 + lane < ncells;
+    float v = 0.f;
+    if (valid && !dead) {
+      const uint32_t sa = tc::smem_u32(slot) + (ss * 32 + lane) * F::CB;
+      const uint32_t ma = tc::smem_u32(slot) + SLOT_CODES + 2 * (ss * 32 + lane);
+      const uint16_t sb = lds16(ma), zb = lds16(ma + F::META);
+      // chunks in an order rotated by the group index: lanes of one shared-memory phase
+      // (consecutive cells) hit different bank groups, and lanes that hold the same group
+      // index (of different rows) read the same activations, which is a broadcast
+      const int rot = BITS == 4 ? (gp >> 1) & 3 : (gp >> 2) & 1;
+      int oc[F::CH], ox[F::CH];
+#pragma unroll
+      for (int c = 0; c < F::CH; ++c) {
+        const int cr = (c + rot) & (F::CH - 1);
+        oc[c] = 16 * cr;
+        ox[c] = 16 * F::UPC * cr;
+      }
+      // the cell's sum carries a factor 2^-24; the scale times 2^24 takes it back (exactly)
+      v = cell_dot<BITS>(sa, xb + 16 * XU * gp, oc, ox, zb) * (__half2float(__ushort_as_half(sb)) * 16777216.f);
+    }
+    // segmented inclusive scan over the lanes of each row within this step
+    const int m = gp < lane ? gp : lane;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, v, off);
+      if (off <= m) v += u;
+    }
+    const float total = gp > lane ? v + carry : v;  // rows begun in an earlier step add the carry
+    if (valid && gp == G - 1 && !dead) y[row] = __half_as_ushort(__float2half_rn(total));
+    const int gp31 = __shfl_sync(0xffffffffu, gp, 31);
+    const float t31 = __shfl_sync(0xffffffffu, total, 31);
+    carry = gp31 == G - 1 ? 0.f : t31;
+    // advance to the cell 32 further on
+    gp += 32;
+    if (G >= 32) {
+      if (gp >= G) {
+        gp -= G;
+        ++row;
+      }
+    } else {
+      const int wr = (int)(((uint32_t)gp * gmul) >> 20);
+      gp -= wr * G;
+      row += wr;
+    }
+    if (ss == F::SPS - 1 || st == nsteps - 1) {  // slot consumed: refill it
+      __syncwarp();
+      ++consumed;
+      if (lane == 0 && !dead) issue(cslot);
+      if (++cslot == slots) {
+        cslot = 0;
+        cphase ^= 1u;
+      }
+    }
+  }
+}
+
+template <int BITS, int CAP>
+__global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant__ StreamParamsT<CAP> P) {
+  using F = Fmt<BITS>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slots = P.slots;
+  uint8_t* ring = smem + (size_t)w * slots * F::SLOT;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)W * slots * F::SLOT) + w * slots;
+  uint8_t* xbase = smem + (size_t)W * slots * (F::SLOT + 8);
+
+  const int64_t share = (P.total_cost + gridDim.x - 1) / gridDim.x;
+  const int64_t lo = share * blockIdx.x, hi = lo + share;
+
+  // first matrix that ends after lo (matrices are in cost order)
+  int mfirst = 0;
+  for (int a = 0, b = P.count; a < b;) {
+    const int c = (a + b) >> 1;
+    if (P.m[c].cost_end <= lo) a = mfirst = c + 1;
+    else b = c;
+  }
+
+  // ---- producer (lane 0 of each warp): the warp's segments, in matrix order, as ring slots
+  Prod pd;
+  pd.cleft = 0;
+  pd.pm = mfirst - 1;
+  int issued = 0, consumed = 0;
+  bool dead = false;  // a bounded wait gave up: stop computing, drain, report
+  auto issue = [&](int slot) {
+    while (pd.cleft == 0) {  // next non-empty segment of this warp
+      if (++pd.pm >= P.count) return;
+      const StreamMat& M = P.m[pd.pm];
+      if (M.cost_begin >= hi) {
+        pd.pm = P.count;
+        return;
+      }
+      int b0, b1;
+      cta_units(M, lo, hi, b0, b1);
+      const Seg sg = warp_seg<BITS>(M, b0, b1, w);
+      pd.c = sg.codes;
+      pd.s = sg.s;
+      pd.z = sg.z;
+      pd.cleft = (int)sg.bytes;
+      pd.gleft = (int)sg.groups;
+    }
+    const uint32_t bar = tc::smem_u32(bars + slot);
+    uint8_t* dst = ring + (size_t)slot * F::SLOT;
+    const int cb = pd.cleft < SLOT_CODES ? pd.cleft : SLOT_CODES;
+    const int gc = pd.gleft < F::GPSL ? pd.gleft : F::GPSL;
+    const uint32_t mb = 2u * (uint32_t)(gc & ~7);  // whole 16-byte units; the rest is done by the consumer
+    tc::mbar_arrive_expect_tx(bar, (uint32_t)cb + 2 * mb);
+    bulk_g2s(tc::smem_u32(dst), pd.c, (uint32_t)cb, bar);
+    if (mb) {
+      bulk_g2s(tc::smem_u32(dst + SLOT_CODES), pd.s, mb, bar);
+      bulk_g2s(tc::smem_u32(dst + SLOT_CODES + F::META), pd.z, mb, bar);
+    }
+    pd.c += cb;
+    pd.s += gc;
+    pd.z += gc;
+    pd.cleft -= cb;
+    pd.gleft -= gc;
+    ++issued;
+  };
+  if (lane == 0) {
+    for (int s = 0; s < slots; ++s) tc::mbar_init(tc::smem_u32(bars + s), 1);
+    tc::fence_mbar_init();
+    for (int s = 0; s < slots; ++s) issue(s);
+  }
+  __syncwarp();
+
+  // ---- consumer
+  int cslot = 0;
+  uint32_t cphase = 0;
+  auto cta_next = [&](int from) -> int {
+    for (int mi = from; mi < P.count; ++mi) {
+      const StreamMat& M = P.m[mi];
+      if (M.cost_begin >= hi) return P.count;
+      if (M.cost_end <= lo) continue;
+      int b0, b1;
+      cta_units(M, lo, hi, b0, b1);
+      if (b0 < b1) return mi;
+    }
+    return P.count;
+  };
+  // activation vector: 16 units of 8 fp16 per group, stored at units 17 g .. 17 g + 15
+  auto stage_x = [&](const StreamMat& M, uint8_t* xb) {
+    const int units = M.K / 8;
+    for (int u = threadIdx.x; u < units; u += T) cp_async16(xb + 16 * (u + (u >> 4)), M.x + 8 * u);
+    cp_async_commit();
+  };
+
+  int mi = cta_next(mfirst);
+  if (P.xbufs == 2 && mi < P.count) stage_x(P.m[mi], xbase);
+  for (int xi = 0; mi < P.count; mi = cta_next(mi + 1), ++xi) {
+    const StreamMat& M = P.m[mi];
+    uint8_t* xb = xbase + (size_t)(P.xbufs == 2 ? (xi & 1) : 0) * P.xbuf_bytes;
+    if (P.xbufs == 1) {
+      __syncthreads();  // everyone is done with the previous vector
+      stage_x(M, xb);
+    }
+    cp_async_wait_all();
+    __syncthreads();  // this matrix's vector is staged; the other buffer is free
+    {
+      const int nx = cta_next(mi + 1);
+      if (nx < P.count) {
+        if (P.xbufs == 2) {
+          stage_x(P.m[nx], xbase + (size_t)((xi + 1) & 1) * P.xbuf_bytes);
+        } else {  // one buffer: have the next vector waiting in L2 when it is staged
+          const int lines = P.m[nx].K / 64;
+          for (int l = threadIdx.x; l < lines; l += T)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(P.m[nx].x + 64 * l));
+        }
+      }
+    }
+    int b0, b1;
+    cta_units(M, lo, hi, b0, b1);
+    const Seg seg = warp_seg<BITS>(M, b0, b1, w);
+    if (seg.rows > 0)
+      consume<BITS>(seg, M, tc::smem_u32(xb), ring, bars, slots, cslot, cphase, consumed, dead, issue, lane);
+  }
+
+  // ---- error path: report, then wait (bounded) for copies still landing in this CTA
+  if (__any_sync(0xffffffffu, dead)) {
+    if (lane == 0) {
+      atomicOr(P.errors, tc::kErrTimeout);
+      for (int j = consumed; j < issued; ++j)
+        tc::mbar_wait(tc::smem_u32(bars + j % slots), (uint32_t)((j / slots) & 1));
+    }
+    __syncwarp();
+  }
+}
+
+int gcd_int(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+template <int BITS>
+int plan_t(StreamParams& p, int count, const StreamDesc* d) {
+  using F = Fmt<BITS>;
+  int64_t cost = 0;
+  int max_k = 0;
+  for (int i = 0; i < count; ++i) {
+    if ((((uintptr_t)d[i].codes | (uintptr_t)d[i].scale | (uintptr_t)d[i].zero | (uintptr_t)d[i].x) & 15) != 0)
+      return 0;
+    const int K = (int)d[i].K, N = (int)d[i].N;
+    const int G = K / kGroup;
+    // rows per unit: segments start at multiples of RA rows, so that their scales and zeros
+    // start on a 16-byte boundary (8 groups)
+    const int RA = 8 / gcd_int(G, 8);
+    const int64_t row_cost = (int64_t)K * BITS / 8 + 4 * G;
+    StreamMat& m = p.m[i];
+    m.codes = d[i].codes;
+    m.scale = d[i].scale;
+    m.zero = d[i].zero;
+    m.x = d[i].x;
+    m.y = d[i].y;
+    m.N = N;
+    m.K = K;
+    m.RA = RA;
+    m.nunit = (N + RA - 1) / RA;
+    m.unit_cost = RA * row_cost;
+    m.cost_begin = cost;
+    cost += (int64_t)N * row_cost;
+    m.cost_end = cost;
+    if (K > max_k) max_k = K;
+  }
+  p.count = count;
+  p.total_cost = cost;
+  p.xbuf_bytes = ((max_k / kGroup) * XU * 16 + 127) & ~127;
+  p.errors = device_error_word();
+  if (!p.errors) return 0;
+  const int options[4][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}};
+  for (const auto& o : options) {
+    const int bytes = W * o[0] * (F::SLOT + 8) + o[1] * p.xbuf_bytes;
+    if (bytes <= kStreamMaxSmem) {
+      p.slots = o[0];
+      p.xbufs = o[1];
+      return bytes;
+    }
+  }
+  return 0;
+}
+
+template <int BITS, int CAP>
+cudaError_t launch_cap(const StreamParamsT<CAP>& p, int smem, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<BITS, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kStreamMaxSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  gemv_stream_kernel<BITS, CAP><<<2 * sms, T, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int BITS, int CAP>
+cudaError_t launch_copy(const StreamParams& p, int smem, cudaStream_t stream) {
+  static thread_local StreamParamsT<CAP> q;
+  q.errors = p.errors;
+  q.total_cost = p.total_cost;
+  q.count = p.count;
+  q.slots = p.slots;
+  q.xbufs = p.xbufs;
+  q.xbuf_bytes = p.xbuf_bytes;
+  for (int i = 0; i < p.count; ++i) q.m[i] = p.m[i];
+  return launch_cap<BITS, CAP>(q, smem, stream);
+}
+
+template <int BITS>
+cudaError_t launch_t(const StreamParams& p, int smem, cudaStream_t stream) {
+  // size the parameter block to the set: a launch copies its whole parameter block
+  if (p.count <= 1) return launch_copy<BITS, 1>(p, smem, stream);
+  if (p.count <= 16) return launch_copy<BITS, 16>(p, smem, stream);
+  if (p.count <= 64) return launch_copy<BITS, 64>(p, smem, stream);
+  return launch_cap<BITS, kStreamMaxMats>(p, smem, stream);
+}
+
+}  // namespace
+
+int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d) {
+  if (count < 1 || count > kStreamMaxMats) return 0;
+  return bits == 4 ? plan_t<4>(p, count, d) : plan_t<2>(p, count, d);
+}
+
+cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int smem, cudaStream_t stream) {
+  return bits == 4 ? launch_t<4>(p, smem, stream) : launch_t<2>(p, smem, stream);
+}
+
+}  // namespace wq

@@ -1,0 +1,57 @@
+// Parameters of the streaming matrix-vector kernel (gemv_stream.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wq {
+
+constexpr int kStreamWarps = 8;              // warps per CTA (two CTAs per SM)
+constexpr int kStreamMaxMats = 256;
+constexpr int kStreamMaxSmem = 113 * 1024;   // per CTA, so that two CTAs fit on one SM
+constexpr int kStreamSlotCodes = 4096;       // bytes of codes per ring slot (one bulk copy)
+
+// One matrix. Rows are dealt to warps in units of RA rows, RA chosen so that every unit's
+// scales and zeros start on a 16-byte boundary; cost counts bytes of codes + scales + zeros.
+struct StreamMat {
+  const void* codes;
+  const uint16_t* scale;
+  const uint16_t* zero;
+  const uint16_t* x;
+  uint16_t* y;
+  int64_t cost_begin;  // cost of the set's matrices before this one
+  int64_t cost_end;    // cost_begin + cost of this matrix
+  int64_t unit_cost;   // cost of one full unit
+  int N, K;
+  int RA;              // rows per unit
+  int nunit;           // ceil(N / RA)
+};
+
+template <int CAP>
+struct StreamParamsT {
+  unsigned int* errors;  // device error word (bounded waits that gave up)
+  int64_t total_cost;
+  int count;
+  int slots;             // ring slots per warp
+  int xbufs;             // staged activation buffers per CTA (1 or 2)
+  int xbuf_bytes;        // bytes of one activation buffer
+  StreamMat m[CAP];
+};
+using StreamParams = StreamParamsT<kStreamMaxMats>;
+
+struct StreamDesc {
+  const void* codes;
+  const uint16_t* scale;
+  const uint16_t* zero;
+  const uint16_t* x;
+  uint16_t* y;
+  int64_t N, K;
+};
+
+// Fills p for a set of `count` matrices of one format (bits 4 or 2) and returns the bytes of
+// dynamic shared memory a CTA needs, or 0 if this kernel cannot serve the set (pointers not
+// 16-byte aligned, or an activation vector too long to stage).
+int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d);
+cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int smem, cudaStream_t stream);
+
+}  // namespace wq

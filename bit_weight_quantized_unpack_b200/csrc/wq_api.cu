@@ -7,6 +7,7 @@
 #include "gemv.cuh"
 #include "gemv_bulk.cuh"
 #include "gemv_rows.cuh"
+#include "gemv_stream.cuh"
 #include "wq.h"
 
 namespace {
@@ -103,6 +104,20 @@ bool plan_bulk(wq::BulkParams& p, int fmt, int count, const wq_linear_desc* d) {
   return true;
 }
 
+// Streaming kernel for a batch-1 set (int4 / int2): needs 16-byte aligned codes, scales,
+// zeros and activations, and activation vectors short enough to stage in shared memory.
+int try_stream(int fmt, int count, const wq_linear_desc* d, cudaStream_t stream, bool* done) {
+  *done = false;
+  if (fmt == WQ_TERNARY || count > wq::kStreamMaxMats) return WQ_OK;
+  static thread_local wq::StreamParams sp;
+  static thread_local wq::StreamDesc sd[wq::kStreamMaxMats];
+  for (int i = 0; i < count; ++i) sd[i] = {d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K};
+  const int smem = wq::stream_plan(sp, fmt == WQ_INT4 ? 4 : 2, count, sd);
+  if (smem == 0) return WQ_OK;
+  *done = true;
+  return cuda_status(wq::launch_gemv_stream(sp, fmt == WQ_INT4 ? 4 : 2, smem, stream));
+}
+
 // Row-per-lane kernel for a batch-1 set (int4 / int2): needs 32-byte aligned codes
 // (its loads are whole 32-byte sectors) and K small enough to stage x in shared memory.
 int try_rows(int fmt, int count, const wq_linear_desc* d, cudaStream_t stream, bool* done) {
@@ -173,7 +188,9 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
   if (M == 1) {
     const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, 1};
     bool done = false;
-    const int r = try_rows(fmt, 1, &d, (cudaStream_t)stream, &done);
+    int r = try_stream(fmt, 1, &d, (cudaStream_t)stream, &done);
+    if (done) return r;
+    r = try_rows(fmt, 1, &d, (cudaStream_t)stream, &done);
     if (done) return r;
   }
   if (M == 1 && fmt != WQ_TERNARY && kUseBulkGemv) {
@@ -251,7 +268,9 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   }
   if (M == 1) {
     bool done = false;
-    const int r = try_rows(fmt, count, descs, (cudaStream_t)stream, &done);
+    int r = try_stream(fmt, count, descs, (cudaStream_t)stream, &done);
+    if (done) return r;
+    r = try_rows(fmt, count, descs, (cudaStream_t)stream, &done);
     if (done) return r;
   }
   if (kUseBulkGemv) {
