@@ -142,19 +142,23 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
-               "l"(gsrc)
-               : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// ceil(num / M.unit_cost) for 0 <= num < 2^52: a double-precision estimate through the
+// stored reciprocal, then an exact integer correction (the estimate is off by at most 1).
+__device__ __forceinline__ int64_t units_ceil(int64_t num, const StreamMat& M) {
+  const int64_t bc = M.unit_cost;
+  int64_t q = (int64_t)((double)num * M.inv_unit_cost);
+  if (q * bc > num) --q;
+  if ((q + 1) * bc <= num) ++q;
+  return q * bc < num ? q + 1 : q;
+}
+
 // Units (RA rows each) of M whose first byte of cost lies in [lo, hi): [b0, b1).
 __device__ __forceinline__ void cta_units(const StreamMat& M, int64_t lo, int64_t hi, int& b0, int& b1) {
-  const int64_t bc = M.unit_cost;
-  const int64_t a = lo <= M.cost_begin ? 0 : (lo - M.cost_begin + bc - 1) / bc;
-  const int64_t b = hi <= M.cost_begin ? 0 : (hi - M.cost_begin + bc - 1) / bc;
+  const int64_t a = lo <= M.cost_begin ? 0 : units_ceil(lo - M.cost_begin, M);
+  const int64_t b = hi <= M.cost_begin ? 0 : units_ceil(hi - M.cost_begin, M);
   b0 = (int)(a < M.nunit ? a : M.nunit);
   b1 = (int)(b < M.nunit ? b : M.nunit);
 }
@@ -166,8 +170,8 @@ struct Seg {
   const uint16_t* z;
   int rows;
   int row0;
-  int64_t bytes;   // codes bytes
-  int64_t groups;  // rows * K / 128
+  int bytes;   // codes bytes
+  int groups;  // rows * K / 128
 };
 
 template <int BITS>
@@ -184,12 +188,13 @@ __device__ __forceinline__ Seg warp_seg(const StreamMat& M, int b0, int b1, int 
   s.codes = reinterpret_cast<const uint8_t*>(M.codes) + r0 * rb;
   s.s = M.scale + r0 * G;
   s.z = M.zero + r0 * G;
-  s.bytes = (int64_t)s.rows * rb;
-  s.groups = (int64_t)s.rows * G;
+  s.bytes = (int)(s.rows * rb);
+  s.groups = s.rows * G;
   return s;
 }
 
-// Copy state of one warp's producer (lane 0): what remains of the current segment.
+// Copy state of one warp's producer, kept identically by all its lanes: what remains of the
+// segment being issued.
 struct Prod {
   const uint8_t* c;
   const uint16_t* s;
@@ -199,15 +204,17 @@ struct Prod {
   int pm;     // matrix of the segment
 };
 
-// Consume one warp segment from the ring: cells in order, lane j taking cell j of each step.
+// Consume one warp segment from the ring: cells in order, lane j taking cell j of each step
+// of 32 cells, SPS steps per ring slot. `issue(slot)` refills a consumed slot (whole warp).
 template <int BITS, class Issue>
-__device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint8_t* ring,
-                                        uint64_t* bars, int slots, int& cslot, uint32_t& cphase, int& consumed,
+__device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint32_t ring,
+                                        uint32_t bars, int slots, int& cslot, uint32_t& cphase, int& consumed,
                                         bool& dead, Issue& issue, int lane) {
   using F = Fmt<BITS>;
   const int G = M.K / kGroup;
-  const int ncells = (int)seg.groups;
+  const int ncells = seg.groups;
   const int nsteps = (ncells + 31) / 32;
+  const int nslots = (nsteps + F::SPS - 1) / F::SPS;
   uint16_t* y = M.y + seg.row0;
   // the matrix's last partial 16-byte unit of scales / zeros, if this segment ends there:
   // loaded now, stored into its ring slot before that slot is read
@@ -219,91 +226,92 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
     if (lane >= 8 && lane < 8 + rem) rz = ld_u16(seg.z + gb + lane - 8);
   }
   // group gp of row `row` of the segment: this lane's cell
-  int gp = lane % G, row = lane / G;
   const uint32_t gmul = ((1u << 20) + G - 1) / G;  // floor(n / G) = (n * gmul) >> 20 for n < G + 32, G < 32
+  int row = G >= 32 ? 0 : (int)(((uint32_t)lane * gmul) >> 20);
+  int gp = lane - row * G;
   float carry = 0.f;  // part of the row that continues from the previous step
-  for (int st = 0; st < nsteps; ++st) {
-    const int ss = st % F::SPS;
-    uint8_t* slot = ring + (size_t)cslot * F::SLOT;
-    if (ss == 0) {
-      if (!dead) {
-        const bool ok = tc::mbar_wait(tc::smem_u32(bars + cslot), cphase);
-        if (!__all_sync(0xffffffffu, ok)) dead = true;
-      }
-      if (rem && (st + F::SPS >= nsteps)) {  // the segment's last slot
-        const int gl = ncells - rem - (st / F::SPS) * F::GPSL;
-        uint16_t* sm = reinterpret_cast<uint16_t*>(slot + SLOT_CODES);
-        if (lane < rem) sm[gl + lane] = rs;
-        if (lane >= 8 && lane < 8 + rem) sm[F::META / 2 + gl + lane - 8] = rz;
-        tc::fence_proxy_async_smem();  // the slot is refilled by bulk copies later
-        __syncwarp();
-      }
+  for (int k = 0; k < nslots; ++k) {
+    const uint32_t slot = ring + cslot * F::SLOT;
+    if (!dead) {
+      const bool ok = tc::mbar_wait(bars + 8 * cslot, cphase);
+      if (!__all_sync(0xffffffffu, ok)) dead = true;
     }
-    const bool valid = st * 32 + lane < ncells;
-    float v = 0.f;
-    if (valid && !dead) {
-      const uint32_t sa = tc::smem_u32(slot) + (ss * 32 + lane) * F::CB;
-      const uint32_t ma = tc::smem_u32(slot) + SLOT_CODES + 2 * (ss * 32 + lane);
-      const uint16_t sb = lds16(ma), zb = lds16(ma + F::META);
-      // chunks in an order rotated by the group index: lanes of one shared-memory phase
-      // (consecutive cells) hit different bank groups, and lanes that hold the same group
-      // index (of different rows) read the same activations, which is a broadcast
-      const int rot = BITS == 4 ? (gp >> 1) & 3 : (gp >> 2) & 1;
-      int oc[F::CH], ox[F::CH];
-#pragma unroll
-      for (int c = 0; c < F::CH; ++c) {
-        const int cr = (c + rot) & (F::CH - 1);
-        oc[c] = 16 * cr;
-        ox[c] = 16 * F::UPC * cr;
-      }
-      // the cell's sum carries a factor 2^-24; the scale times 2^24 takes it back (exactly)
-      v = cell_dot<BITS>(sa, xb + 16 * XU * gp, oc, ox, zb) * (__half2float(__ushort_as_half(sb)) * 16777216.f);
-    }
-    // segmented inclusive scan over the lanes of each row within this step
-    const int m = gp < lane ? gp : lane;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float u = __shfl_up_sync(0xffffffffu, v, off);
-      if (off <= m) v += u;
-    }
-    const float total = gp > lane ? v + carry : v;  // rows begun in an earlier step add the carry
-    if (valid && gp == G - 1 && !dead) y[row] = __half_as_ushort(__float2half_rn(total));
-    const int gp31 = __shfl_sync(0xffffffffu, gp, 31);
-    const float t31 = __shfl_sync(0xffffffffu, total, 31);
-    carry = gp31 == G - 1 ? 0.f : t31;
-    // advance to the cell 32 further on
-    gp += 32;
-    if (G >= 32) {
-      if (gp >= G) {
-        gp -= G;
-        ++row;
-      }
-    } else {
-      const int wr = (int)(((uint32_t)gp * gmul) >> 20);
-      gp -= wr * G;
-      row += wr;
-    }
-    if (ss == F::SPS - 1 || st == nsteps - 1) {  // slot consumed: refill it
+    if (rem && k == nslots - 1) {
+      const int gl = ncells - rem - k * F::GPSL;
+      if (lane < rem) asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + SLOT_CODES + 2 * (gl + lane)), "h"(rs));
+      if (lane >= 8 && lane < 8 + rem)
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + SLOT_CODES + F::META + 2 * (gl + lane - 8)), "h"(rz));
+      tc::fence_proxy_async_smem();  // the slot is refilled by bulk copies later
       __syncwarp();
-      ++consumed;
-      if (lane == 0 && !dead) issue(cslot);
-      if (++cslot == slots) {
-        cslot = 0;
-        cphase ^= 1u;
+    }
+    const uint32_t cell0 = slot + lane * F::CB, meta0 = slot + SLOT_CODES + 2 * lane;
+#pragma unroll
+    for (int ss = 0; ss < F::SPS; ++ss) {
+      const int st = k * F::SPS + ss;
+      if (F::SPS > 1 && st >= nsteps) break;
+      const bool valid = st * 32 + lane < ncells;
+      float v = 0.f;
+      if (valid && !dead) {
+        const uint16_t sb = lds16(meta0 + 64 * ss), zb = lds16(meta0 + 64 * ss + F::META);
+        // chunks in an order permuted by the group index: lanes of one shared-memory phase
+        // (consecutive cells) hit different bank groups, and lanes that hold the same group
+        // index (of different rows) read the same activations, which is a broadcast
+        const int rot = BITS == 4 ? (gp >> 1) & 3 : (gp >> 2) & 1;
+        int oc[F::CH], ox[F::CH];
+#pragma unroll
+        for (int c = 0; c < F::CH; ++c) {
+          oc[c] = 16 * (c ^ rot);
+          ox[c] = 16 * F::UPC * (c ^ rot);
+        }
+        // the cell's sum carries a factor 2^-24; the scale times 2^24 takes it back (exactly)
+        v = cell_dot<BITS>(cell0 + 32 * F::CB * ss, xb + 16 * XU * gp, oc, ox, zb) *
+            (__half2float(__ushort_as_half(sb)) * 16777216.f);
       }
+      // segmented inclusive scan over the lanes of each row within this step
+      const int m = gp < lane ? gp : lane;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, off);
+        if (off <= m) v += u;
+      }
+      const float total = gp > lane ? v + carry : v;  // rows begun in an earlier step add the carry
+      if (valid && gp == G - 1 && !dead) y[row] = __half_as_ushort(__float2half_rn(total));
+      const int gp31 = __shfl_sync(0xffffffffu, gp, 31);
+      const float t31 = __shfl_sync(0xffffffffu, total, 31);
+      carry = gp31 == G - 1 ? 0.f : t31;
+      // advance to the cell 32 further on
+      gp += 32;
+      if (G >= 32) {
+        if (gp >= G) {
+          gp -= G;
+          ++row;
+        }
+      } else {
+        const int wr = (int)(((uint32_t)gp * gmul) >> 20);
+        gp -= wr * G;
+        row += wr;
+      }
+    }
+    __syncwarp();  // every lane is done reading the slot: refill it
+    ++consumed;
+    if (!dead) issue(cslot);
+    if (++cslot == slots) {
+      cslot = 0;
+      cphase ^= 1u;
     }
   }
 }
 
 template <int BITS, int CAP>
-__global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant__ StreamParamsT<CAP> P) {
+__global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(const __grid_constant__ StreamParamsT<CAP> P) {
   using F = Fmt<BITS>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slots = P.slots;
-  uint8_t* ring = smem + (size_t)w * slots * F::SLOT;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)W * slots * F::SLOT) + w * slots;
-  uint8_t* xbase = smem + (size_t)W * slots * (F::SLOT + 8);
+  const uint32_t sbase = tc::smem_u32(smem);
+  const uint32_t ring = sbase + w * slots * F::SLOT;
+  const uint32_t bars = sbase + W * slots * F::SLOT + 8 * w * slots;
+  const uint32_t xbase = sbase + W * slots * (F::SLOT + 8);
 
   const int64_t share = (P.total_cost + gridDim.x - 1) / gridDim.x;
   const int64_t lo = share * blockIdx.x, hi = lo + share;
@@ -316,7 +324,8 @@ __global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant
     else b = c;
   }
 
-  // ---- producer (lane 0 of each warp): the warp's segments, in matrix order, as ring slots
+  // ---- producer: the warp's segments, in matrix order, as ring slots (state kept by every
+  // lane alike; lanes 0, 1, 2 issue the codes, scales and zeros copies of a slot together)
   Prod pd;
   pd.cleft = 0;
   pd.pm = mfirst - 1;
@@ -336,19 +345,21 @@ __global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant
       pd.c = sg.codes;
       pd.s = sg.s;
       pd.z = sg.z;
-      pd.cleft = (int)sg.bytes;
-      pd.gleft = (int)sg.groups;
+      pd.cleft = sg.bytes;
+      pd.gleft = sg.groups;
     }
-    const uint32_t bar = tc::smem_u32(bars + slot);
-    uint8_t* dst = ring + (size_t)slot * F::SLOT;
-    const int cb = pd.cleft < SLOT_CODES ? pd.cleft : SLOT_CODES;
-    const int gc = pd.gleft < F::GPSL ? pd.gleft : F::GPSL;
+    const uint32_t bar = bars + 8 * slot, dst = ring + slot * F::SLOT;
+    int cb = SLOT_CODES, gc = F::GPSL;
+    if (pd.cleft < SLOT_CODES) {
+      cb = pd.cleft;
+      gc = pd.gleft;
+    }
     const uint32_t mb = 2u * (uint32_t)(gc & ~7);  // whole 16-byte units; the rest is done by the consumer
-    tc::mbar_arrive_expect_tx(bar, (uint32_t)cb + 2 * mb);
-    bulk_g2s(tc::smem_u32(dst), pd.c, (uint32_t)cb, bar);
-    if (mb) {
-      bulk_g2s(tc::smem_u32(dst + SLOT_CODES), pd.s, mb, bar);
-      bulk_g2s(tc::smem_u32(dst + SLOT_CODES + F::META), pd.z, mb, bar);
+    if (lane == 0) tc::mbar_arrive_expect_tx(bar, (uint32_t)cb + 2 * mb);
+    if (lane == 0 || (lane < 3 && mb)) {
+      const void* src = lane == 0 ? (const void*)pd.c : lane == 1 ? (const void*)pd.s : (const void*)pd.z;
+      const uint32_t d = lane == 0 ? dst : dst + SLOT_CODES + (lane - 1) * F::META;
+      bulk_g2s(d, src, lane == 0 ? (uint32_t)cb : mb, bar);
     }
     pd.c += cb;
     pd.s += gc;
@@ -358,11 +369,11 @@ __global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant
     ++issued;
   };
   if (lane == 0) {
-    for (int s = 0; s < slots; ++s) tc::mbar_init(tc::smem_u32(bars + s), 1);
+    for (int s = 0; s < slots; ++s) tc::mbar_init(bars + 8 * s, 1);
     tc::fence_mbar_init();
-    for (int s = 0; s < slots; ++s) issue(s);
   }
   __syncwarp();
+  for (int s = 0; s < slots; ++s) issue(s);
 
   // ---- consumer
   int cslot = 0;
@@ -379,9 +390,11 @@ __global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant
     return P.count;
   };
   // activation vector: 16 units of 8 fp16 per group, stored at units 17 g .. 17 g + 15
-  auto stage_x = [&](const StreamMat& M, uint8_t* xb) {
+  auto stage_x = [&](const StreamMat& M, uint32_t xb) {
     const int units = M.K / 8;
-    for (int u = threadIdx.x; u < units; u += T) cp_async16(xb + 16 * (u + (u >> 4)), M.x + 8 * u);
+    for (int u = threadIdx.x; u < units; u += T)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + 16 * (u + (u >> 4))), "l"(M.x + 8 * u)
+                   : "memory");
     cp_async_commit();
   };
 
@@ -389,7 +402,7 @@ __global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant
   if (P.xbufs == 2 && mi < P.count) stage_x(P.m[mi], xbase);
   for (int xi = 0; mi < P.count; mi = cta_next(mi + 1), ++xi) {
     const StreamMat& M = P.m[mi];
-    uint8_t* xb = xbase + (size_t)(P.xbufs == 2 ? (xi & 1) : 0) * P.xbuf_bytes;
+    const uint32_t xb = xbase + (P.xbufs == 2 ? (xi & 1) : 0) * P.xbuf_bytes;
     if (P.xbufs == 1) {
       __syncthreads();  // everyone is done with the previous vector
       stage_x(M, xb);
@@ -400,7 +413,7 @@ __global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant
       const int nx = cta_next(mi + 1);
       if (nx < P.count) {
         if (P.xbufs == 2) {
-          stage_x(P.m[nx], xbase + (size_t)((xi + 1) & 1) * P.xbuf_bytes);
+          stage_x(P.m[nx], xbase + ((xi + 1) & 1) * P.xbuf_bytes);
         } else {  // one buffer: have the next vector waiting in L2 when it is staged
           const int lines = P.m[nx].K / 64;
           for (int l = threadIdx.x; l < lines; l += T)
@@ -411,16 +424,14 @@ __global__ void __launch_bounds__(T, 2) gemv_stream_kernel(const __grid_constant
     int b0, b1;
     cta_units(M, lo, hi, b0, b1);
     const Seg seg = warp_seg<BITS>(M, b0, b1, w);
-    if (seg.rows > 0)
-      consume<BITS>(seg, M, tc::smem_u32(xb), ring, bars, slots, cslot, cphase, consumed, dead, issue, lane);
+    if (seg.rows > 0) consume<BITS>(seg, M, xb, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane);
   }
 
   // ---- error path: report, then wait (bounded) for copies still landing in this CTA
   if (__any_sync(0xffffffffu, dead)) {
     if (lane == 0) {
       atomicOr(P.errors, tc::kErrTimeout);
-      for (int j = consumed; j < issued; ++j)
-        tc::mbar_wait(tc::smem_u32(bars + j % slots), (uint32_t)((j / slots) & 1));
+      for (int j = consumed; j < issued; ++j) tc::mbar_wait(bars + 8 * (j % slots), (uint32_t)((j / slots) & 1));
     }
     __syncwarp();
   }
@@ -460,6 +471,7 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d) {
     m.RA = RA;
     m.nunit = (N + RA - 1) / RA;
     m.unit_cost = RA * row_cost;
+    m.inv_unit_cost = 1.0 / (double)m.unit_cost;
     m.cost_begin = cost;
     cost += (int64_t)N * row_cost;
     m.cost_end = cost;
@@ -470,16 +482,17 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d) {
   p.xbuf_bytes = ((max_k / kGroup) * XU * 16 + 127) & ~127;
   p.errors = device_error_word();
   if (!p.errors) return 0;
-  const int options[4][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}};
-  for (const auto& o : options) {
-    const int bytes = W * o[0] * (F::SLOT + 8) + o[1] * p.xbuf_bytes;
-    if (bytes <= kStreamMaxSmem) {
-      p.slots = o[0];
-      p.xbufs = o[1];
-      return bytes;
-    }
-  }
-  return 0;
+  // two ring slots per warp; two activation buffers when four CTAs still fit on an SM
+  // (measured best on the 0.5B decode set), else one; then as many CTAs as fit
+  const int ring = W * 2 * (F::SLOT + 8);
+  const int two = ring + 2 * p.xbuf_bytes, one = ring + p.xbuf_bytes;
+  const int bytes = (kStreamSmPool / (two + 1024) >= kStreamMaxCtasPerSm) ? two : one;
+  if (bytes > kStreamMaxSmem) return 0;
+  p.slots = 2;
+  p.xbufs = bytes == two ? 2 : 1;
+  const int fit = kStreamSmPool / (bytes + 1024);
+  p.ctas_per_sm = fit < kStreamMaxCtasPerSm ? fit : kStreamMaxCtasPerSm;
+  return bytes;
 }
 
 template <int BITS, int CAP>
@@ -497,7 +510,7 @@ cudaError_t launch_cap(const StreamParamsT<CAP>& p, int smem, cudaStream_t strea
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  gemv_stream_kernel<BITS, CAP><<<2 * sms, T, smem, stream>>>(p);
+  gemv_stream_kernel<BITS, CAP><<<p.ctas_per_sm * sms, T, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -509,6 +522,7 @@ cudaError_t launch_copy(const StreamParams& p, int smem, cudaStream_t stream) {
   q.count = p.count;
   q.slots = p.slots;
   q.xbufs = p.xbufs;
+  q.ctas_per_sm = p.ctas_per_sm;
   q.xbuf_bytes = p.xbuf_bytes;
   for (int i = 0; i < p.count; ++i) q.m[i] = p.m[i];
   return launch_cap<BITS, CAP>(q, smem, stream);

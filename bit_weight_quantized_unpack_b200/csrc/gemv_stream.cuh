@@ -6,9 +6,11 @@
 
 namespace wq {
 
-constexpr int kStreamWarps = 8;              // warps per CTA (two CTAs per SM)
+constexpr int kStreamWarps = 4;              // warps per CTA (up to four CTAs per SM)
+constexpr int kStreamMaxCtasPerSm = 4;       // register budget of the launch bounds
 constexpr int kStreamMaxMats = 256;
-constexpr int kStreamMaxSmem = 113 * 1024;   // per CTA, so that two CTAs fit on one SM
+constexpr int kStreamSmPool = 233472;        // shared memory of one SM (228 KB)
+constexpr int kStreamMaxSmem = 232448;       // per CTA (227 KB)
 constexpr int kStreamSlotCodes = 4096;       // bytes of codes per ring slot (one bulk copy)
 
 // One matrix. Rows are dealt to warps in units of RA rows, RA chosen so that every unit's
@@ -22,6 +24,7 @@ struct StreamMat {
   int64_t cost_begin;  // cost of the set's matrices before this one
   int64_t cost_end;    // cost_begin + cost of this matrix
   int64_t unit_cost;   // cost of one full unit
+  double inv_unit_cost;  // 1 / unit_cost
   int N, K;
   int RA;              // rows per unit
   int nunit;           // ceil(N / RA)
@@ -34,6 +37,7 @@ struct StreamParamsT {
   int count;
   int slots;             // ring slots per warp
   int xbufs;             // staged activation buffers per CTA (1 or 2)
+  int ctas_per_sm;       // CTAs that fit on one SM with this set's shared memory
   int xbuf_bytes;        // bytes of one activation buffer
   StreamMat m[CAP];
 };
