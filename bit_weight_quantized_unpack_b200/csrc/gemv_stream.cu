@@ -9,10 +9,11 @@
 //
 // The staged bytes are a stream of cells, one cell = one row's 128-weight group (64 bytes
 // of int4 codes, 32 of int2). Lane j takes cell j of each step of 32 cells. Its 16-byte
-// chunks are read in an order rotated by the cell's group index, so that the eight lanes of
-// a shared-memory phase hit eight different bank groups and lanes holding the same group
-// index read the same activations (a broadcast); the activation vector is staged with 17
-// units of 16 bytes per group (one spare) for the same reason.
+// chunks are read in an order permuted by the cell's group index, so that the eight lanes
+// of a shared-memory phase hit eight different bank groups; the activation vector is staged
+// with each group's chunks in that same order and 17 units of 16 bytes per group (one
+// spare), so that activation reads are conflict-free too, and lanes holding the same group
+// index read the same activations (a broadcast).
 //
 // Dequantisation is one AND per pair of codes: the masked bits of a binary16 lane are the
 // subnormal number q * 2^-24 (16 q * 2^-24 for the high nibble of a byte, which stays below
@@ -40,6 +41,13 @@ constexpr int W = kStreamWarps;
 constexpr int T = 32 * W;
 constexpr int SLOT_CODES = kStreamSlotCodes;
 constexpr int XU = 17;  // staged activation units (16 bytes) per 128-weight group
+
+// Chunk permutation of group g (XOR mask on the chunk index), shared by the codes reads and
+// the staged activation layout.
+template <int BITS>
+__host__ __device__ __forceinline__ int xrot(int g) {
+  return BITS == 4 ? (g >> 1) & 3 : (g >> 2) & 1;
+}
 
 template <int BITS>
 struct Fmt {
@@ -253,15 +261,17 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
       float v = 0.f;
       if (valid && !dead) {
         const uint16_t sb = lds16(meta0 + 64 * ss), zb = lds16(meta0 + 64 * ss + F::META);
-        // chunks in an order permuted by the group index: lanes of one shared-memory phase
-        // (consecutive cells) hit different bank groups, and lanes that hold the same group
-        // index (of different rows) read the same activations, which is a broadcast
-        const int rot = BITS == 4 ? (gp >> 1) & 3 : (gp >> 2) & 1;
+        // chunks in an order permuted by the group index, so that the lanes of one
+        // shared-memory phase (consecutive cells) hit different bank groups; the staged
+        // activations of each group are stored in that same order (see stage_x), so the
+        // x chunk read at step c is always the c-th stored one, and lanes that hold the same
+        // group index (of different rows) read the same activations, which is a broadcast
+        const int rot = xrot<BITS>(gp);
         int oc[F::CH], ox[F::CH];
 #pragma unroll
         for (int c = 0; c < F::CH; ++c) {
           oc[c] = 16 * (c ^ rot);
-          ox[c] = 16 * F::UPC * (c ^ rot);
+          ox[c] = 16 * F::UPC * c;
         }
         // the cell's sum carries a factor 2^-24; the scale times 2^24 takes it back (exactly)
         v = cell_dot<BITS>(cell0 + 32 * F::CB * ss, xb + 16 * XU * gp, oc, ox, zb) *
@@ -389,12 +399,15 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     }
     return P.count;
   };
-  // activation vector: 16 units of 8 fp16 per group, stored at units 17 g .. 17 g + 15
+  // activation vector: the 16 units (8 fp16 each) of group g at units 17 g .. 17 g + 15,
+  // its chunks (UPC units each) in the order of the group's chunk permutation
   auto stage_x = [&](const StreamMat& M, uint32_t xb) {
     const int units = M.K / 8;
-    for (int u = threadIdx.x; u < units; u += T)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + 16 * (u + (u >> 4))), "l"(M.x + 8 * u)
-                   : "memory");
+    for (int u = threadIdx.x; u < units; u += T) {
+      const int g = u >> 4, lc = (u & 15) / F::UPC, i = u & (F::UPC - 1);
+      const int pu = XU * g + F::UPC * (lc ^ xrot<BITS>(g)) + i;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + 16 * pu), "l"(M.x + 8 * u) : "memory");
+    }
     cp_async_commit();
   };
 
