@@ -32,6 +32,9 @@ from bit_weight_quantized_unpack_b200 import synth, workloads  # noqa: E402
 
 METRIC = "int4 g128 batch-1 GEMV weight GB/s (% of HBM peak); M=512 GEMM TFLOPS"
 INT4_BYTES_PER_WEIGHT = 0.5 + 4 / 128  # codes + fp16 scale + fp16 zero per 128 weights
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gemv_stream_kernel launch
+# over the 0.5B decode set, from one ncu capture of the current kernel (None once it changes)
+GEMV_TRAFFIC_BYTES = 263553280 + 5531648
 
 
 def peaks():
@@ -312,7 +315,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(nbytes / ms / 1e6, 2),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(nbytes / ms / 1e6 / pk["hbm_gbs"], 4),
-                         "traffic": None, "kernel": "gemv_stream_kernel<4, 256>",
+                         "traffic": GEMV_TRAFFIC_BYTES, "kernel": "gemv_stream_kernel<4, 256>",
                          "peak_source": pk["source"]},
             "e2e": {"value": round(nbytes * ws / ms_e2e / 1e6, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * K_tot, "d2h_bytes_per_step": 2 * N_tot},

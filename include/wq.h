@@ -34,7 +34,9 @@
  *                                   group = sum_{i<5} (t_{5j+i} + 1) * 3^i; byte 25 holds
  *                                   trits 125..127 and two pad trits 0 (digit 1); every
  *                                   byte is in 0..242
- *   scale, zero  fp16 bits (uint16) [N, G]; zero is unused (NULL) for WQ_TERNARY
+ *   scale, zero  fp16 bits (uint16) [N, G]; zero is unused (NULL) for WQ_TERNARY; a zero
+ *                point is an integer in [0, 2^b - 1] (as wq_quantize writes it); the
+ *                kernels use its nearest integer
  *   x, X, y, Y   fp16 bits (uint16), X [M, K] and Y [M, N] row-major
  *
  * Conventions.
