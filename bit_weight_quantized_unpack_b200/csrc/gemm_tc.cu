@@ -103,21 +103,6 @@ __device__ __forceinline__ uint4 dequant8(uint32_t v, uint32_t c1024z, uint32_t 
   return r;
 }
 
-// First tile whose starting cost is >= target (tiles of all matrices numbered in order).
-template <int CAP>
-__device__ int first_tile_at(const TcParamsT<CAP>& P, int64_t target) {
-  for (int i = 0; i < P.count; ++i) {
-    const TcMat& m = P.m[i];
-    const int64_t end = m.cost_begin + (int64_t)(m.tile_end - m.tile_begin) * m.tile_cost;
-    if (target < end) {
-      const int64_t off = target - m.cost_begin;
-      const int64_t j = off <= 0 ? 0 : (off + m.tile_cost - 1) / m.tile_cost;
-      return m.tile_begin + (int)j;
-    }
-  }
-  return P.total_tiles;
-}
-
 struct SzPair {
   uint16_t s, z;  // fp16 bits of one group's scale and zero
 };
@@ -142,8 +127,7 @@ __device__ __forceinline__ TileInfo tile_info(const TcParamsT<CAP>& P, int tile,
 
 }  // namespace
 
-// Persistent: CTA b runs the tiles whose starting cost lies in its 1/gridDim share, in
-// order. Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31 = weight rows), 4 TMA producer,
+// Persistent: CTA b runs tiles b, b + gridDim.x, ... in order. Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31 = weight rows), 4 TMA producer,
 // 5 MMA issuer (and TMEM owner), 8-15 dequantisers (two threads per weight row, 32 k each
 // per stage); 6-7 idle. The two 256-column TMEM accumulators let the epilogue of one tile
 // overlap the main loop of the next.
@@ -188,9 +172,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   tc::tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  const int64_t share = (P.total_cost + gridDim.x - 1) / gridDim.x;
-  const int t_lo = first_tile_at(P, share * blockIdx.x);
-  const int t_hi = first_tile_at(P, share * (blockIdx.x + 1));
+  // tiles are dealt to CTAs round robin (CTA b takes tiles b, b + gridDim.x, ...); the host
+  // orders each launch's matrices by tile cost, largest first, so every CTA gets the same mix
+  const int t_lo = blockIdx.x, t_step = gridDim.x, t_hi = P.total_tiles;
 
   bool timed_out = false;
   int it = 0;    // k-block sequence number over this CTA's tiles
@@ -199,7 +183,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   if (warp == XPROD_WARP) {
     // activation tiles, one per k-block
     if (lane == 0) {
-      for (int tile = t_lo; tile < t_hi && !timed_out; ++tile) {
+      for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step) {
         const TileInfo ti = tile_info(P, tile, mi);
         const TcMat& M = P.m[ti.mi];
         const uint32_t tx = (uint32_t)(ti.bn * BK * 2);
@@ -215,7 +199,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   } else if (warp == MMA_WARP) {
     if (lane == 0) {
       int lt = 0;
-      for (int tile = t_lo; tile < t_hi && !timed_out; ++tile, ++lt) {
+      for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step, ++lt) {
         const TileInfo ti = tile_info(P, tile, mi);
         const int b = lt & 1;
         if (!tc::mbar_wait(bar_tempty + 8 * b, ((lt >> 1) & 1) ^ 1)) { timed_out = true; break; }
@@ -269,7 +253,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
       c.kb += 2;
       if (c.kb >= c.ti.nkb) {
         c.kb = team;
-        if (++c.tile < t_hi) c.ti = tile_info(P, c.tile, c.mi);
+        c.tile += t_step;
+        if (c.tile < t_hi) c.ti = tile_info(P, c.tile, c.mi);
       }
     };
     // Codes are not copied by TMA: a slow DRAM copy would hold up the activation copies
@@ -309,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     sz0 = sz_fetch();
     sz1 = sz_fetch();
     int cseq = 0;
-    for (int tile = t_lo; tile < t_hi && !timed_out; ++tile) {
+    for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step) {
       const TileInfo ti = tile_info(P, tile, mi);
       for (int kb = team; kb < ti.nkb; kb += 2) {
         const int itk = it + kb;               // sequence number of this k-block
@@ -346,7 +331,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     int lt = 0, nst = 0;
     const uint32_t ebuf = sbase + OFF_E + (uint32_t)(warp * 2 * EPI_BYTES);
     uint16_t* ebuf_g = reinterpret_cast<uint16_t*>(smem + OFF_E + warp * 2 * EPI_BYTES);
-    for (int tile = t_lo; tile < t_hi && !timed_out; ++tile, ++lt) {
+    for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step, ++lt) {
       const TileInfo ti = tile_info(P, tile, mi);
       const TcMat& M = P.m[ti.mi];
       const int b = lt & 1;

@@ -240,14 +240,27 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   if (fmt == WQ_INT4 && M >= wq::kTcMinM) {
     // tensor-core GEMM: persistent launches of up to kTcMaxMats matrices each
     static thread_local wq::TcParams tp;
-    // as few launches as the parameter block allows, with equal matrix counts
+    // as few launches as the parameter block allows. Matrices are ordered by the cost of
+    // their tiles (K), largest first, and dealt to the launches round robin, so that every
+    // launch, whose CTAs take its tiles round robin, ends with small tiles on all SMs.
     const int launches = (count + wq::kTcMaxMats - 1) / wq::kTcMaxMats;
-    for (int l = 0, i0 = 0; l < launches; ++l) {
-      const int n = (count - i0) / (launches - l);
+    static thread_local int order[WQ_LINEAR_SET_MAX];
+    for (int i = 0; i < count; ++i) order[i] = i;
+    for (int i = 1; i < count; ++i) {  // stable insertion sort by K, descending
+      const int v = order[i];
+      int j = i;
+      while (j > 0 && descs[order[j - 1]].K < descs[v].K) {
+        order[j] = order[j - 1];
+        --j;
+      }
+      order[j] = v;
+    }
+    for (int l = 0; l < launches; ++l) {
+      const int n = (count - l + launches - 1) / launches;  // matrices l, l + launches, ...
       int tiles = 0;
       int64_t cost = 0;
       for (int j = 0; j < n; ++j) {
-        const wq_linear_desc& d = descs[i0 + j];
+        const wq_linear_desc& d = descs[order[l + j * launches]];
         wq::TcMat& t = tp.m[j];
         if (!wq::tc_plan_mat(t, d.x, (int)M, d.codes, d.scale, d.zero, d.y, (int)d.N, (int)d.K, wq::tc_bn_for((int)M)))
           return WQ_ERR_CUDA;
@@ -262,7 +275,6 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
       tp.total_cost = cost;
       const int st = cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
       if (st != WQ_OK) return st;
-      i0 += n;
     }
     return WQ_OK;
   }
