@@ -231,7 +231,8 @@ def bench_rows(args, pk):
 
 def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 64, 512, 2048)):
     """Batch sweep on the 0.5B set: M tokens through all 169 matrices in one wq_linear_set
-    call per pass (tensor-core launches of up to 80 matrices for M >= 16)."""
+    call per pass (one streaming launch for M <= 4; tensor-core launches of up to 80
+    matrices for M >= 5)."""
     from bit_weight_quantized_unpack_b200 import wq
     wl = workloads.WORKLOADS[4]
     mats = workloads.workload_mats(4)
@@ -259,7 +260,7 @@ def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 64, 512, 2048)):
         out[f"gemm_set_M{M}"] = {"ms": ms, "TFLOPS": flops / ms / 1e9,
                                  "frac_tensor": flops / ms / 1e9 / pk["bf16_tflops"],
                                  "weight_GBps": weights * INT4_BYTES_PER_WEIGHT / ms / 1e6,
-                                 "launches_per_pass": (len(mats) + 79) // 80 if M >= 16 else 1}
+                                 "launches_per_pass": (len(mats) + 79) // 80 if M >= 5 else 1}
         del X, Y
         torch.cuda.empty_cache()
     return out

@@ -71,12 +71,14 @@ __device__ __forceinline__ uint16_t lds16(uint32_t a) {
   return v;
 }
 
-// Dot products of one 16-byte chunk of codes with its activations (shared-memory address
-// xa), accumulated in binary32 with the factor 2^-24 described above.
-// int4: 32 codes; z1 / z16 hold z and 16 z as binary16 bit patterns in both lanes; the A
-// accumulators take codes at bits 0-3 of a byte, the B ones (16x) bits 4-7.
-__device__ __forceinline__ void chunk_int4(const uint4 c, uint32_t xa, uint32_t z1, uint32_t z16, float& a0,
-                                           float& a1, float& b0, float& b1) {
+// Dot products of one 16-byte chunk of codes with the activations of MT rows of X (row m
+// at shared-memory address xa + m * xs), accumulated in binary32 with the factor 2^-24
+// described above. Each pair of codes is dequantised once for all MT rows.
+// int4: 32 codes; z1 / z16 hold z and 16 z as binary16 bit patterns in both lanes; the a
+// accumulators take codes at bits 0-3 of a byte, the b ones (16x) bits 4-7.
+template <int MT>
+__device__ __forceinline__ void chunk_int4(const uint4 c, uint32_t xa, uint32_t xs, uint32_t z1, uint32_t z16,
+                                           float (&a)[MT][2], float (&b)[MT][2]) {
   const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -85,62 +87,80 @@ __device__ __forceinline__ void chunk_int4(const uint4 c, uint32_t xa, uint32_t 
     const uint32_t d1 = hsub2_u32(v & 0x00F000F0u, z16);   // 16 q1, 16 q5
     const uint32_t d2 = hsub2_u32(v8 & 0x000F000Fu, z1);   // q2, q6
     const uint32_t d3 = hsub2_u32(v8 & 0x00F000F0u, z16);  // 16 q3, 16 q7
-    const uint4 xw = lds128(xa + 16 * i);  // (x0, x1) (x2, x3) (x4, x5) (x6, x7)
-    float& A = (i & 1) ? a1 : a0;
-    float& B = (i & 1) ? b1 : b0;
-    A = fma_f16f16_f32(lo16(d0), lo16(xw.x), A);
-    A = fma_f16f16_f32(hi16(d0), lo16(xw.z), A);
-    A = fma_f16f16_f32(lo16(d2), lo16(xw.y), A);
-    A = fma_f16f16_f32(hi16(d2), lo16(xw.w), A);
-    B = fma_f16f16_f32(lo16(d1), hi16(xw.x), B);
-    B = fma_f16f16_f32(hi16(d1), hi16(xw.z), B);
-    B = fma_f16f16_f32(lo16(d3), hi16(xw.y), B);
-    B = fma_f16f16_f32(hi16(d3), hi16(xw.w), B);
-  }
-}
-
-// int2: 64 codes (four words of 16); zm[m] holds 4^m z as binary16 bits in both lanes; the
-// lanes of d are codes j and j + 8 of a word, scaled by 4^(j mod 4), accumulated in a[j mod 4].
-__device__ __forceinline__ void chunk_int2(const uint4 c, uint32_t xa, const uint32_t (&zm)[4], float (&a)[4]) {
-  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t v = cw[i], v8 = v >> 8;
-    const uint4 xl = lds128(xa + 32 * i), xh = lds128(xa + 32 * i + 16);  // x0 .. x7, x8 .. x15
-    const uint32_t xlw[4] = {xl.x, xl.y, xl.z, xl.w}, xhw[4] = {xh.x, xh.y, xh.z, xh.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t d = hsub2_u32((j < 4 ? v : v8) & (0x00030003u << (2 * (j & 3))), zm[j & 3]);
-      const uint16_t xj = (j & 1) ? hi16(xlw[j >> 1]) : lo16(xlw[j >> 1]);
-      const uint16_t xj8 = (j & 1) ? hi16(xhw[j >> 1]) : lo16(xhw[j >> 1]);
-      a[j & 3] = fma_f16f16_f32(lo16(d), xj, a[j & 3]);
-      a[j & 3] = fma_f16f16_f32(hi16(d), xj8, a[j & 3]);
+    for (int m = 0; m < MT; ++m) {
+      const uint4 xw = lds128(xa + m * xs + 16 * i);  // (x0, x1) (x2, x3) (x4, x5) (x6, x7)
+      float& A = a[m][i & 1];
+      float& B = b[m][i & 1];
+      A = fma_f16f16_f32(lo16(d0), lo16(xw.x), A);
+      A = fma_f16f16_f32(hi16(d0), lo16(xw.z), A);
+      A = fma_f16f16_f32(lo16(d2), lo16(xw.y), A);
+      A = fma_f16f16_f32(hi16(d2), lo16(xw.w), A);
+      B = fma_f16f16_f32(lo16(d1), hi16(xw.x), B);
+      B = fma_f16f16_f32(hi16(d1), hi16(xw.z), B);
+      B = fma_f16f16_f32(lo16(d3), hi16(xw.y), B);
+      B = fma_f16f16_f32(hi16(d3), hi16(xw.w), B);
     }
   }
 }
 
-// 2^-24 * sum_k x_k (q_k - z) over one cell at shared address `cell`; xg: shared address of
-// the group's activation units; oc[c] / ox[c]: offsets of the cell's c-th chunk in this
-// lane's rotated order and of that chunk's first activation unit.
-template <int BITS>
-__device__ __forceinline__ float cell_dot(uint32_t cell, uint32_t xg, const int (&oc)[Fmt<BITS>::CH],
-                                          const int (&ox)[Fmt<BITS>::CH], uint16_t zbits) {
+// int2: 64 codes (four words of 16); zm[k] holds 4^k z as binary16 bits in both lanes; the
+// lanes of d_j are codes j and j + 8 of a word, scaled by 4^(j mod 4), accumulated in
+// a[m][j mod 4].
+template <int MT>
+__device__ __forceinline__ void chunk_int2(const uint4 c, uint32_t xa, uint32_t xs, const uint32_t (&zm)[4],
+                                           float (&a)[MT][4]) {
+  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t v = cw[i], v8 = v >> 8;
+    uint32_t d[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) d[j] = hsub2_u32((j < 4 ? v : v8) & (0x00030003u << (2 * (j & 3))), zm[j & 3]);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const uint4 xl = lds128(xa + m * xs + 32 * i), xh = lds128(xa + m * xs + 32 * i + 16);  // x0..x7, x8..x15
+      const uint32_t xlw[4] = {xl.x, xl.y, xl.z, xl.w}, xhw[4] = {xh.x, xh.y, xh.z, xh.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint16_t xj = (j & 1) ? hi16(xlw[j >> 1]) : lo16(xlw[j >> 1]);
+        const uint16_t xj8 = (j & 1) ? hi16(xhw[j >> 1]) : lo16(xhw[j >> 1]);
+        a[m][j & 3] = fma_f16f16_f32(lo16(d[j]), xj, a[m][j & 3]);
+        a[m][j & 3] = fma_f16f16_f32(hi16(d[j]), xj8, a[m][j & 3]);
+      }
+    }
+  }
+}
+
+// out[m] = 2^-24 * sum_k x_mk (q_k - z) over one cell at shared address `cell`, for the MT
+// rows of X; xg: shared address of the group's activation units in row 0, xs: bytes between
+// rows; oc[c] / ox[c]: offsets of the cell's c-th chunk in this lane's permuted order and of
+// that chunk's first activation unit.
+template <int BITS, int MT>
+__device__ __forceinline__ void cell_dot(uint32_t cell, uint32_t xg, uint32_t xs, const int (&oc)[Fmt<BITS>::CH],
+                                         const int (&ox)[Fmt<BITS>::CH], uint16_t zbits, float (&out)[MT]) {
   using F = Fmt<BITS>;
   const uint32_t zi = (uint32_t)__half2int_rn(__ushort_as_half(zbits));  // integer zero point
   if constexpr (BITS == 4) {
     const uint32_t z1 = zi * 0x00010001u, z16 = zi * 0x00100010u;
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+    float a[MT][2], b[MT][2];
 #pragma unroll
-    for (int c = 0; c < F::CH; ++c) chunk_int4(lds128(cell + oc[c]), xg + ox[c], z1, z16, a0, a1, b0, b1);
-    return fmaf(b0 + b1, 0.0625f, a0 + a1);
+    for (int m = 0; m < MT; ++m) a[m][0] = a[m][1] = b[m][0] = b[m][1] = 0.f;
+#pragma unroll
+    for (int c = 0; c < F::CH; ++c) chunk_int4<MT>(lds128(cell + oc[c]), xg + ox[c], xs, z1, z16, a, b);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) out[m] = fmaf(b[m][0] + b[m][1], 0.0625f, a[m][0] + a[m][1]);
   } else {
     uint32_t zm[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) zm[m] = (zi << (2 * m)) * 0x00010001u;
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < 4; ++k) zm[k] = (zi << (2 * k)) * 0x00010001u;
+    float a[MT][4];
 #pragma unroll
-    for (int c = 0; c < F::CH; ++c) chunk_int2(lds128(cell + oc[c]), xg + ox[c], zm, a);
-    return fmaf(a[3], 0.015625f, fmaf(a[2], 0.0625f, fmaf(a[1], 0.25f, a[0])));
+    for (int m = 0; m < MT; ++m) a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0.f;
+#pragma unroll
+    for (int c = 0; c < F::CH; ++c) chunk_int2<MT>(lds128(cell + oc[c]), xg + ox[c], xs, zm, a);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) out[m] = fmaf(a[m][3], 0.015625f, fmaf(a[m][2], 0.0625f, fmaf(a[m][1], 0.25f, a[m][0])));
   }
 }
 
@@ -214,7 +234,7 @@ struct Prod {
 
 // Consume one warp segment from the ring: cells in order, lane j taking cell j of each step
 // of 32 cells, SPS steps per ring slot. `issue(slot)` refills a consumed slot (whole warp).
-template <int BITS, class Issue>
+template <int BITS, int MT, class Issue>
 __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint32_t ring,
                                         uint32_t bars, int slots, int& cslot, uint32_t& cphase, int& consumed,
                                         bool& dead, Issue& issue, int lane) {
@@ -237,7 +257,10 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
   const uint32_t gmul = ((1u << 20) + G - 1) / G;  // floor(n / G) = (n * gmul) >> 20 for n < G + 32, G < 32
   int row = G >= 32 ? 0 : (int)(((uint32_t)lane * gmul) >> 20);
   int gp = lane - row * G;
-  float carry = 0.f;  // part of the row that continues from the previous step
+  const uint32_t xs = (uint32_t)(G * XU * 16);  // bytes between the staged rows of X
+  float carry[MT];  // per row of X: part of the row of W that continues from the previous step
+#pragma unroll
+  for (int m = 0; m < MT; ++m) carry[m] = 0.f;
   for (int k = 0; k < nslots; ++k) {
     const uint32_t slot = ring + cslot * F::SLOT;
     if (!dead) {
@@ -258,7 +281,9 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
       const int st = k * F::SPS + ss;
       if (F::SPS > 1 && st >= nsteps) break;
       const bool valid = st * 32 + lane < ncells;
-      float v = 0.f;
+      float v[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) v[m] = 0.f;
       if (valid && !dead) {
         const uint16_t sb = lds16(meta0 + 64 * ss), zb = lds16(meta0 + 64 * ss + F::META);
         // chunks in an order permuted by the group index, so that the lanes of one
@@ -274,21 +299,29 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
           ox[c] = 16 * F::UPC * c;
         }
         // the cell's sum carries a factor 2^-24; the scale times 2^24 takes it back (exactly)
-        v = cell_dot<BITS>(cell0 + 32 * F::CB * ss, xb + 16 * XU * gp, oc, ox, zb) *
-            (__half2float(__ushort_as_half(sb)) * 16777216.f);
+        cell_dot<BITS, MT>(cell0 + 32 * F::CB * ss, xb + 16 * XU * gp, xs, oc, ox, zb, v);
+        const float s24 = __half2float(__ushort_as_half(sb)) * 16777216.f;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) v[m] *= s24;
       }
       // segmented inclusive scan over the lanes of each row within this step
-      const int m = gp < lane ? gp : lane;
+      const int lim = gp < lane ? gp : lane;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, v, off);
-        if (off <= m) v += u;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float u = __shfl_up_sync(0xffffffffu, v[m], off);
+          if (off <= lim) v[m] += u;
+        }
       }
-      const float total = gp > lane ? v + carry : v;  // rows begun in an earlier step add the carry
-      if (valid && gp == G - 1 && !dead) y[row] = __half_as_ushort(__float2half_rn(total));
       const int gp31 = __shfl_sync(0xffffffffu, gp, 31);
-      const float t31 = __shfl_sync(0xffffffffu, total, 31);
-      carry = gp31 == G - 1 ? 0.f : t31;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const float total = gp > lane ? v[m] + carry[m] : v[m];  // rows begun earlier add the carry
+        if (valid && gp == G - 1 && !dead) y[(size_t)m * M.N + row] = __half_as_ushort(__float2half_rn(total));
+        const float t31 = __shfl_sync(0xffffffffu, total, 31);
+        carry[m] = gp31 == G - 1 ? 0.f : t31;
+      }
       // advance to the cell 32 further on
       gp += 32;
       if (G >= 32) {
@@ -312,7 +345,7 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
   }
 }
 
-template <int BITS, int CAP>
+template <int BITS, int MT, int CAP>
 __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(const __grid_constant__ StreamParamsT<CAP> P) {
   using F = Fmt<BITS>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -399,14 +432,17 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     }
     return P.count;
   };
-  // activation vector: the 16 units (8 fp16 each) of group g at units 17 g .. 17 g + 15,
-  // its chunks (UPC units each) in the order of the group's chunk permutation
+  // activations, row by row of X: the 16 units (8 fp16 each) of group g at units
+  // 17 g .. 17 g + 15 of the row, its chunks (UPC units each) in the order of the group's
+  // chunk permutation
   auto stage_x = [&](const StreamMat& M, uint32_t xb) {
-    const int units = M.K / 8;
-    for (int u = threadIdx.x; u < units; u += T) {
+    const int units = M.K / 8, rowu = (M.K / kGroup) * XU;
+    for (int t = threadIdx.x; t < MT * units; t += T) {
+      const int m = t / units, u = t - m * units;
       const int g = u >> 4, lc = (u & 15) / F::UPC, i = u & (F::UPC - 1);
-      const int pu = XU * g + F::UPC * (lc ^ xrot<BITS>(g)) + i;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + 16 * pu), "l"(M.x + 8 * u) : "memory");
+      const int pu = m * rowu + XU * g + F::UPC * (lc ^ xrot<BITS>(g)) + i;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + 16 * pu), "l"(M.x + (size_t)8 * t)
+                   : "memory");
     }
     cp_async_commit();
   };
@@ -428,7 +464,7 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
         if (P.xbufs == 2) {
           stage_x(P.m[nx], xbase + ((xi + 1) & 1) * P.xbuf_bytes);
         } else {  // one buffer: have the next vector waiting in L2 when it is staged
-          const int lines = P.m[nx].K / 64;
+          const int lines = MT * P.m[nx].K / 64;
           for (int l = threadIdx.x; l < lines; l += T)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(P.m[nx].x + 64 * l));
         }
@@ -437,7 +473,7 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     int b0, b1;
     cta_units(M, lo, hi, b0, b1);
     const Seg seg = warp_seg<BITS>(M, b0, b1, w);
-    if (seg.rows > 0) consume<BITS>(seg, M, xb, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane);
+    if (seg.rows > 0) consume<BITS, MT>(seg, M, xb, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane);
   }
 
   // ---- error path: report, then wait (bounded) for copies still landing in this CTA
@@ -460,7 +496,7 @@ int gcd_int(int a, int b) {
 }
 
 template <int BITS>
-int plan_t(StreamParams& p, int count, const StreamDesc* d) {
+int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   using F = Fmt<BITS>;
   int64_t cost = 0;
   int max_k = 0;
@@ -492,7 +528,7 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d) {
   }
   p.count = count;
   p.total_cost = cost;
-  p.xbuf_bytes = ((max_k / kGroup) * XU * 16 + 127) & ~127;
+  p.xbuf_bytes = (mt * (max_k / kGroup) * XU * 16 + 127) & ~127;
   p.errors = device_error_word();
   if (!p.errors) return 0;
   // two ring slots per warp; two activation buffers when four CTAs still fit on an SM
@@ -508,11 +544,11 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d) {
   return bytes;
 }
 
-template <int BITS, int CAP>
+template <int BITS, int MT, int CAP>
 cudaError_t launch_cap(const StreamParamsT<CAP>& p, int smem, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<BITS, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<BITS, MT, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kStreamMaxSmem);
     if (e != cudaSuccess) return e;
     configured = true;
@@ -523,11 +559,11 @@ cudaError_t launch_cap(const StreamParamsT<CAP>& p, int smem, cudaStream_t strea
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  gemv_stream_kernel<BITS, CAP><<<p.ctas_per_sm * sms, T, smem, stream>>>(p);
+  gemv_stream_kernel<BITS, MT, CAP><<<p.ctas_per_sm * sms, T, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <int BITS, int CAP>
+template <int BITS, int MT, int CAP>
 cudaError_t launch_copy(const StreamParams& p, int smem, cudaStream_t stream) {
   static thread_local StreamParamsT<CAP> q;
   q.errors = p.errors;
@@ -538,27 +574,36 @@ cudaError_t launch_copy(const StreamParams& p, int smem, cudaStream_t stream) {
   q.ctas_per_sm = p.ctas_per_sm;
   q.xbuf_bytes = p.xbuf_bytes;
   for (int i = 0; i < p.count; ++i) q.m[i] = p.m[i];
-  return launch_cap<BITS, CAP>(q, smem, stream);
+  return launch_cap<BITS, MT, CAP>(q, smem, stream);
+}
+
+template <int BITS, int MT>
+cudaError_t launch_t(const StreamParams& p, int smem, cudaStream_t stream) {
+  // size the parameter block to the set: a launch copies its whole parameter block
+  if (p.count <= 1) return launch_copy<BITS, MT, 1>(p, smem, stream);
+  if (MT == 1 && p.count <= 64) return launch_copy<BITS, MT, 64>(p, smem, stream);
+  return launch_cap<BITS, MT, kStreamMaxMats>(p, smem, stream);
 }
 
 template <int BITS>
-cudaError_t launch_t(const StreamParams& p, int smem, cudaStream_t stream) {
-  // size the parameter block to the set: a launch copies its whole parameter block
-  if (p.count <= 1) return launch_copy<BITS, 1>(p, smem, stream);
-  if (p.count <= 16) return launch_copy<BITS, 16>(p, smem, stream);
-  if (p.count <= 64) return launch_copy<BITS, 64>(p, smem, stream);
-  return launch_cap<BITS, kStreamMaxMats>(p, smem, stream);
+cudaError_t launch_b(const StreamParams& p, int mt, int smem, cudaStream_t stream) {
+  switch (mt) {
+    case 1: return launch_t<BITS, 1>(p, smem, stream);
+    case 2: return launch_t<BITS, 2>(p, smem, stream);
+    case 3: return launch_t<BITS, 3>(p, smem, stream);
+    default: return launch_t<BITS, 4>(p, smem, stream);
+  }
 }
 
 }  // namespace
 
-int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d) {
-  if (count < 1 || count > kStreamMaxMats) return 0;
-  return bits == 4 ? plan_t<4>(p, count, d) : plan_t<2>(p, count, d);
+int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int mt) {
+  if (count < 1 || count > kStreamMaxMats || mt < 1 || mt > kStreamMaxRows) return 0;
+  return bits == 4 ? plan_t<4>(p, count, d, mt) : plan_t<2>(p, count, d, mt);
 }
 
-cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int smem, cudaStream_t stream) {
-  return bits == 4 ? launch_t<4>(p, smem, stream) : launch_t<2>(p, smem, stream);
+cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem, cudaStream_t stream) {
+  return bits == 4 ? launch_b<4>(p, mt, smem, stream) : launch_b<2>(p, mt, smem, stream);
 }
 
 }  // namespace wq

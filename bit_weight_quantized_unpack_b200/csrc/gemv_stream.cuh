@@ -9,6 +9,7 @@ namespace wq {
 constexpr int kStreamWarps = 4;              // warps per CTA (up to four CTAs per SM)
 constexpr int kStreamMaxCtasPerSm = 4;       // register budget of the launch bounds
 constexpr int kStreamMaxMats = 256;
+constexpr int kStreamMaxRows = 4;            // rows of X per product (M = 1 .. 4)
 constexpr int kStreamSmPool = 233472;        // shared memory of one SM (228 KB)
 constexpr int kStreamMaxSmem = 232448;       // per CTA (227 KB)
 constexpr int kStreamSlotCodes = 4096;       // bytes of codes per ring slot (one bulk copy)
@@ -52,10 +53,11 @@ struct StreamDesc {
   int64_t N, K;
 };
 
-// Fills p for a set of `count` matrices of one format (bits 4 or 2) and returns the bytes of
-// dynamic shared memory a CTA needs, or 0 if this kernel cannot serve the set (pointers not
-// 16-byte aligned, or an activation vector too long to stage).
-int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d);
-cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int smem, cudaStream_t stream);
+// Fills p for a set of `count` matrices of one format (bits 4 or 2), each multiplied by mt
+// rows of X (X [mt, K] and Y [mt, N] row-major), and returns the bytes of dynamic shared
+// memory a CTA needs, or 0 if this kernel cannot serve the set (pointers not 16-byte
+// aligned, or activations too long to stage).
+int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int mt);
+cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem, cudaStream_t stream);
 
 }  // namespace wq

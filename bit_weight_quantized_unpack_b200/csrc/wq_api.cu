@@ -104,18 +104,20 @@ bool plan_bulk(wq::BulkParams& p, int fmt, int count, const wq_linear_desc* d) {
   return true;
 }
 
-// Streaming kernel for a batch-1 set (int4 / int2): needs 16-byte aligned codes, scales,
-// zeros and activations, and activation vectors short enough to stage in shared memory.
-int try_stream(int fmt, int count, const wq_linear_desc* d, cudaStream_t stream, bool* done) {
+// Streaming kernel for a set (int4 / int2) with M = 1 .. 4 rows of X: needs 16-byte aligned
+// codes, scales, zeros and activations, and activations short enough to stage in shared
+// memory.
+int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStream_t stream, bool* done) {
   *done = false;
-  if (fmt == WQ_TERNARY || count > wq::kStreamMaxMats) return WQ_OK;
+  if (fmt == WQ_TERNARY || count > wq::kStreamMaxMats || M > wq::kStreamMaxRows) return WQ_OK;
   static thread_local wq::StreamParams sp;
   static thread_local wq::StreamDesc sd[wq::kStreamMaxMats];
   for (int i = 0; i < count; ++i) sd[i] = {d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K};
-  const int smem = wq::stream_plan(sp, fmt == WQ_INT4 ? 4 : 2, count, sd);
+  const int bits = fmt == WQ_INT4 ? 4 : 2;
+  const int smem = wq::stream_plan(sp, bits, count, sd, (int)M);
   if (smem == 0) return WQ_OK;
   *done = true;
-  return cuda_status(wq::launch_gemv_stream(sp, fmt == WQ_INT4 ? 4 : 2, smem, stream));
+  return cuda_status(wq::launch_gemv_stream(sp, bits, (int)M, smem, stream));
 }
 
 // Row-per-lane kernel for a batch-1 set (int4 / int2): needs 32-byte aligned codes
@@ -185,13 +187,15 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
     tp.total_cost = (int64_t)tp.total_tiles * tp.m[0].tile_cost;
     return cuda_status(wq::launch_gemm_tc(tp, (cudaStream_t)stream));
   }
-  if (M == 1) {
-    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, 1};
+  if (M <= wq::kStreamMaxRows) {
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, M};
     bool done = false;
-    int r = try_stream(fmt, 1, &d, (cudaStream_t)stream, &done);
+    int r = try_stream(fmt, 1, &d, M, (cudaStream_t)stream, &done);
     if (done) return r;
-    r = try_rows(fmt, 1, &d, (cudaStream_t)stream, &done);
-    if (done) return r;
+    if (M == 1) {
+      r = try_rows(fmt, 1, &d, (cudaStream_t)stream, &done);
+      if (done) return r;
+    }
   }
   if (M == 1 && fmt != WQ_TERNARY && kUseBulkGemv) {
     static thread_local wq::BulkParams bp;
@@ -278,12 +282,14 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
     }
     return WQ_OK;
   }
-  if (M == 1) {
+  if (M <= wq::kStreamMaxRows) {
     bool done = false;
-    int r = try_stream(fmt, count, descs, (cudaStream_t)stream, &done);
+    int r = try_stream(fmt, count, descs, M, (cudaStream_t)stream, &done);
     if (done) return r;
-    r = try_rows(fmt, count, descs, (cudaStream_t)stream, &done);
-    if (done) return r;
+    if (M == 1) {
+      r = try_rows(fmt, count, descs, (cudaStream_t)stream, &done);
+      if (done) return r;
+    }
   }
   if (kUseBulkGemv) {
     static thread_local wq::BulkParams bp;
