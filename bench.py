@@ -223,6 +223,17 @@ def bench_rows(args, pk):
         ms = time_steps(step, 200 if not args.quick else 20, 10, 1)
         rows[f"gemv_lm_head_{fmt}"] = {"ms": ms, "GBps": nb / ms / 1e6,
                                        "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"]}
+        if fmt == "int4":
+            # fused greedy pick: product and argmax in one launch, y not stored
+            ws = torch.zeros(wq.wq_argmax_workspace_bytes(), dtype=torch.uint8, device="cuda")
+            am = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+            def step_am(i, copies=copies):
+                c, s, z = copies[i % len(copies)]
+                wq.wq_gemv_argmax(x, c, s, z, "int4", N, K, None, am, ws, ws.numel())
+            ms = time_steps(step_am, 200 if not args.quick else 20, 10, 1)
+            rows["gemv_argmax_lm_head_int4"] = {"ms": ms, "GBps": nb / ms / 1e6,
+                                                "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"]}
         del copies
         torch.cuda.empty_cache()
     rows.update(bench_batch_sweep(args, pk))

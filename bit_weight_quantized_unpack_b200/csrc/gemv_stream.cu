@@ -28,6 +28,9 @@
 //
 // The activation vector of the matrix being processed is staged once per CTA; two buffers
 // let the next matrix's vector load while the current one is in use.
+#include <climits>
+#include <cmath>
+
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_stream.cuh"
@@ -234,10 +237,12 @@ struct Prod {
 
 // Consume one warp segment from the ring: cells in order, lane j taking cell j of each step
 // of 32 cells, SPS steps per ring slot. `issue(slot)` refills a consumed slot (whole warp).
-template <int BITS, int MT, class Issue>
+// AM: also keep this lane's best (fp16 value, row) among the rows it completes, for the fused
+// argmax (ties to the lowest row).
+template <int BITS, int MT, bool AM, class Issue>
 __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint32_t ring,
                                         uint32_t bars, int slots, int& cslot, uint32_t& cphase, int& consumed,
-                                        bool& dead, Issue& issue, int lane) {
+                                        bool& dead, Issue& issue, int lane, float& bv, int& bi) {
   using F = Fmt<BITS>;
   const int G = M.K / kGroup;
   const int ncells = seg.groups;
@@ -318,7 +323,18 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         const float total = gp > lane ? v[m] + carry[m] : v[m];  // rows begun earlier add the carry
-        if (valid && gp == G - 1 && !dead) y[(size_t)m * M.N + row] = __half_as_ushort(__float2half_rn(total));
+        if (valid && gp == G - 1 && !dead) {
+          const __half h = __float2half_rn(total);
+          if (M.y) y[(size_t)m * M.N + row] = __half_as_ushort(h);
+          if (AM) {
+            const float hv = __half2float(h);
+            const int r = seg.row0 + row;
+            if (hv > bv || (hv == bv && r < bi)) {
+              bv = hv;
+              bi = r;
+            }
+          }
+        }
         const float t31 = __shfl_sync(0xffffffffu, total, 31);
         carry[m] = gp31 == G - 1 ? 0.f : t31;
       }
@@ -345,7 +361,15 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
   }
 }
 
-template <int BITS, int MT, int CAP>
+// Better of two (value, row) candidates of the fused argmax: larger value, then lower row.
+__device__ __forceinline__ void am_take(float& bv, int& bi, float v, int i) {
+  if (v > bv || (v == bv && i < bi)) {
+    bv = v;
+    bi = i;
+  }
+}
+
+template <int BITS, int MT, int CAP, bool AM>
 __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(const __grid_constant__ StreamParamsT<CAP> P) {
   using F = Fmt<BITS>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -447,6 +471,8 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     cp_async_commit();
   };
 
+  float am_v = -INFINITY;  // fused argmax: this lane's best fp16 value and its row
+  int am_i = INT_MAX;
   int mi = cta_next(mfirst);
   if (P.xbufs == 2 && mi < P.count) stage_x(P.m[mi], xbase);
   for (int xi = 0; mi < P.count; mi = cta_next(mi + 1), ++xi) {
@@ -473,7 +499,57 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     int b0, b1;
     cta_units(M, lo, hi, b0, b1);
     const Seg seg = warp_seg<BITS>(M, b0, b1, w);
-    if (seg.rows > 0) consume<BITS, MT>(seg, M, xb, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane);
+    if (seg.rows > 0)
+      consume<BITS, MT, AM>(seg, M, xb, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane, am_v, am_i);
+  }
+
+  // ---- fused argmax: warp, CTA, then the last CTA to finish combines every CTA's partial
+  // (each CTA publishes its partial, fences, takes a ticket; the holder of the last ticket
+  // reads them all and resets the ticket counter for the next call)
+  if (AM) {
+    __shared__ float s_v[W];
+    __shared__ int s_i[W];
+    __shared__ int s_last;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      am_take(am_v, am_i, __shfl_xor_sync(0xffffffffu, am_v, off), __shfl_xor_sync(0xffffffffu, am_i, off));
+    if (lane == 0) {
+      s_v[w] = am_v;
+      s_i[w] = am_i;
+    }
+    __syncthreads();
+    float* part = reinterpret_cast<float*>(P.am_ws + 4);
+    if (threadIdx.x == 0) {
+      float v = s_v[0];
+      int i = s_i[0];
+      for (int k = 1; k < W; ++k) am_take(v, i, s_v[k], s_i[k]);
+      part[2 * blockIdx.x] = v;
+      reinterpret_cast<int*>(part)[2 * blockIdx.x + 1] = i;
+      __threadfence();
+      s_last = atomicAdd(P.am_ws, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      float v = -INFINITY;
+      int i = INT_MAX;
+      for (int b = threadIdx.x; b < (int)gridDim.x; b += T)
+        am_take(v, i, __ldcg(part + 2 * b), __ldcg(reinterpret_cast<const int*>(part) + 2 * b + 1));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        am_take(v, i, __shfl_xor_sync(0xffffffffu, v, off), __shfl_xor_sync(0xffffffffu, i, off));
+      __syncthreads();  // s_v / s_i are reused
+      if (lane == 0) {
+        s_v[w] = v;
+        s_i[w] = i;
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        for (int k = 1; k < W; ++k) am_take(s_v[0], s_i[0], s_v[k], s_i[k]);
+        *P.am_out = s_i[0];
+        *P.am_ws = 0u;  // ticket counter back to zero for the next call
+      }
+    }
   }
 
   // ---- error path: report, then wait (bounded) for copies still landing in this CTA
@@ -528,6 +604,8 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   }
   p.count = count;
   p.total_cost = cost;
+  p.am_ws = nullptr;
+  p.am_out = nullptr;
   p.xbuf_bytes = (mt * (max_k / kGroup) * XU * 16 + 127) & ~127;
   p.errors = device_error_word();
   if (!p.errors) return 0;
@@ -544,28 +622,34 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   return bytes;
 }
 
-template <int BITS, int MT, int CAP>
-cudaError_t launch_cap(const StreamParamsT<CAP>& p, int smem, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<BITS, MT, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kStreamMaxSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+int sm_count() {
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  gemv_stream_kernel<BITS, MT, CAP><<<p.ctas_per_sm * sms, T, smem, stream>>>(p);
+  return sms;
+}
+
+template <int BITS, int MT, int CAP, bool AM = false>
+cudaError_t launch_cap(const StreamParamsT<CAP>& p, int smem, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<BITS, MT, CAP, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kStreamMaxSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  gemv_stream_kernel<BITS, MT, CAP, AM><<<p.ctas_per_sm * sm_count(), T, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <int BITS, int MT, int CAP>
+template <int BITS, int MT, int CAP, bool AM = false>
 cudaError_t launch_copy(const StreamParams& p, int smem, cudaStream_t stream) {
   static thread_local StreamParamsT<CAP> q;
+  q.am_ws = p.am_ws;
+  q.am_out = p.am_out;
   q.errors = p.errors;
   q.total_cost = p.total_cost;
   q.count = p.count;
@@ -574,7 +658,7 @@ cudaError_t launch_copy(const StreamParams& p, int smem, cudaStream_t stream) {
   q.ctas_per_sm = p.ctas_per_sm;
   q.xbuf_bytes = p.xbuf_bytes;
   for (int i = 0; i < p.count; ++i) q.m[i] = p.m[i];
-  return launch_cap<BITS, MT, CAP>(q, smem, stream);
+  return launch_cap<BITS, MT, CAP, AM>(q, smem, stream);
 }
 
 template <int BITS, int MT>
@@ -605,5 +689,11 @@ int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int m
 cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem, cudaStream_t stream) {
   return bits == 4 ? launch_b<4>(p, mt, smem, stream) : launch_b<2>(p, mt, smem, stream);
 }
+
+cudaError_t launch_gemv_stream_argmax(const StreamParams& p, int bits, int smem, cudaStream_t stream) {
+  return bits == 4 ? launch_copy<4, 1, 1, true>(p, smem, stream) : launch_copy<2, 1, 1, true>(p, smem, stream);
+}
+
+int stream_grid(const StreamParams& p) { return p.ctas_per_sm * sm_count(); }
 
 }  // namespace wq

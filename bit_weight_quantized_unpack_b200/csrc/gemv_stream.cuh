@@ -11,7 +11,7 @@ constexpr int kStreamMaxCtasPerSm = 4;       // register budget of the launch bo
 constexpr int kStreamMaxMats = 256;
 constexpr int kStreamMaxRows = 4;            // rows of X per product (M = 1 .. 4)
 constexpr int kStreamSmPool = 233472;        // shared memory of one SM (228 KB)
-constexpr int kStreamMaxSmem = 232448;       // per CTA (227 KB)
+constexpr int kStreamMaxSmem = 232448 - 1024; // dynamic, per CTA (227 KB less room for static)
 constexpr int kStreamSlotCodes = 4096;       // bytes of codes per ring slot (one bulk copy)
 
 // One matrix. Rows are dealt to warps in units of RA rows, RA chosen so that every unit's
@@ -40,6 +40,11 @@ struct StreamParamsT {
   int xbufs;             // staged activation buffers per CTA (1 or 2)
   int ctas_per_sm;       // CTAs that fit on one SM with this set's shared memory
   int xbuf_bytes;        // bytes of one activation buffer
+  // fused argmax over the rows of a single matrix (null when not wanted): work space of
+  // 16 + 8 * gridDim.x bytes whose first word is a CTA ticket counter (zero between calls),
+  // followed by one (fp32 value, int32 row) partial per CTA; the result row goes to am_out
+  unsigned int* am_ws;
+  int* am_out;
   StreamMat m[CAP];
 };
 using StreamParams = StreamParamsT<kStreamMaxMats>;
@@ -59,5 +64,10 @@ struct StreamDesc {
 // aligned, or activations too long to stage).
 int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int mt);
 cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem, cudaStream_t stream);
+// One matrix (p.count == 1, mt == 1) with the fused argmax of its fp16 outputs (ties to the
+// lowest row); p.am_ws / p.am_out must be set. Grid = p.ctas_per_sm * SMs CTAs.
+cudaError_t launch_gemv_stream_argmax(const StreamParams& p, int bits, int smem, cudaStream_t stream);
+// CTAs the streaming kernel launches for a plan (the argmax work space holds one partial each).
+int stream_grid(const StreamParams& p);
 
 }  // namespace wq

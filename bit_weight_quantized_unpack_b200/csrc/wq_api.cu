@@ -306,6 +306,37 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   return cuda_status(wq::launch_gemv_set(p, fmt, (int)M, (cudaStream_t)stream));
 }
 
+size_t wq_argmax_workspace_bytes(void) {
+  if (check_device() != WQ_OK) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return 16 + 8 * (size_t)wq::kStreamMaxCtasPerSm * (size_t)sms;
+}
+
+int wq_gemv_argmax(const uint16_t* x, const void* codes, const uint16_t* scale, const uint16_t* zero, int fmt,
+                   int64_t N, int64_t K, uint16_t* y, int32_t* argmax, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  int st = check_shape(fmt, N, K);
+  if (st != WQ_OK) return st;
+  if (fmt == WQ_TERNARY || !x || !argmax || !workspace) return WQ_ERR_ARG;
+  if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scale, 16) || !aligned(zero, 16) ||
+      !aligned(workspace, 16) || (y && !aligned(y, 2)) || !aligned(argmax, 4))
+    return WQ_ERR_ALIGN;
+  if (K > 32768) return WQ_ERR_SHAPE;
+  if ((st = check_device()) != WQ_OK) return st;
+  static thread_local wq::StreamParams sp;
+  const wq::StreamDesc d = {codes, scale, zero, x, y, N, K};
+  const int bits = fmt == WQ_INT4 ? 4 : 2;
+  const int smem = wq::stream_plan(sp, bits, 1, &d, 1);
+  if (smem == 0) return WQ_ERR_SHAPE;
+  if (workspace_bytes < 16 + 8 * (size_t)wq::stream_grid(sp)) return WQ_ERR_ARG;
+  sp.am_ws = static_cast<unsigned int*>(workspace);
+  sp.am_out = reinterpret_cast<int*>(argmax);
+  return cuda_status(wq::launch_gemv_stream_argmax(sp, bits, smem, (cudaStream_t)stream));
+}
+
 const char* wq_status_str(int status) {
   switch (status) {
     case WQ_OK: return "WQ_OK";

@@ -43,6 +43,8 @@ _sig = {
     "wq_status_str": (ctypes.c_char_p, [_i]),
     "wq_last_cuda_error": (_i, []),
     "wq_device_errors": (_i, [ctypes.POINTER(ctypes.c_uint), _i, _p]),
+    "wq_argmax_workspace_bytes": (ctypes.c_size_t, []),
+    "wq_gemv_argmax": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p, _p, ctypes.c_size_t, _p]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -104,6 +106,18 @@ def wq_gemv(x, codes, scale, zero, fmt, N, K, y, stream=None) -> None:
 def wq_gemm(X, M, codes, scale, zero, fmt, N, K, Y, stream=None) -> None:
     _check(_lib.wq_gemm(_ptr(X), M, _ptr(codes), _ptr(scale), _ptr(zero), _fmt(fmt), N, K,
                         _ptr(Y), _stream(stream)), "wq_gemm")
+
+
+def wq_argmax_workspace_bytes() -> int:
+    return _lib.wq_argmax_workspace_bytes()
+
+
+def wq_gemv_argmax(x, codes, scale, zero, fmt, N, K, y, argmax, workspace, workspace_bytes,
+                   stream=None) -> None:
+    """y may be None; argmax is a device int32 tensor; workspace a zero-filled device buffer."""
+    _check(_lib.wq_gemv_argmax(_ptr(x), _ptr(codes), _ptr(scale), _ptr(zero), _fmt(fmt), N, K,
+                               _ptr(y), _ptr(argmax), _ptr(workspace), workspace_bytes,
+                               _stream(stream)), "wq_gemv_argmax")
 
 
 def make_linear_set(entries) -> ctypes.Array:

@@ -128,6 +128,28 @@ typedef struct {
  * M. 1 <= count <= WQ_LINEAR_SET_MAX; each entry obeys the wq_gemm requirements. */
 int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream);
 
+/* Bytes of device work space wq_gemv_argmax needs on the current device (one 8-byte partial
+ * per CTA of its launch plus a 16-byte header); 0 if no supported device is current. */
+size_t wq_argmax_workspace_bytes(void);
+
+/* Greedy pick fused into the output-projection product: y = x . w_hat^T exactly as wq_gemv
+ * computes it (fp16, rounded once), and *argmax = the row n with the largest y[n], compared
+ * as fp16 values, ties to the lowest n -- in one launch, with no read-back of y (Whetstone
+ * README, notes on --temperature 0: greedy decoding stays on the GPU because the argmax is
+ * written where the next step reads it).
+ *   fmt        WQ_INT4 or WQ_INT2 (WQ_ERR_ARG otherwise).
+ *   y          device fp16 [N], or NULL to skip storing the outputs.
+ *   argmax     device int32, written with the row index.
+ *   workspace  device buffer of at least wq_argmax_workspace_bytes() bytes, 16-byte aligned,
+ *              zero-filled by the caller before its first use; every call leaves its first
+ *              4 bytes zero again. Two calls that share a work space must not overlap on the
+ *              GPU (same stream, or ordered by events).
+ * codes, scale, zero and x must be 16-byte aligned (WQ_ERR_ALIGN) and K at most 32768
+ * (WQ_ERR_SHAPE); other requirements as for wq_gemv. Inputs must be finite. */
+int wq_gemv_argmax(const uint16_t* x, const void* codes, const uint16_t* scale,
+                   const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* y,
+                   int32_t* argmax, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static string naming a status code. */
 const char* wq_status_str(int status);
 
