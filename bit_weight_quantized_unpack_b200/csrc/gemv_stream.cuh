@@ -69,5 +69,7 @@ cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem
 cudaError_t launch_gemv_stream_argmax(const StreamParams& p, int bits, int smem, cudaStream_t stream);
 // CTAs the streaming kernel launches for a plan (the argmax work space holds one partial each).
 int stream_grid(const StreamParams& p);
+// Records e as the library's last CUDA error (wq_last_cuda_error); returns the wq_status.
+int note_cuda_error(cudaError_t e);
 
 }  // namespace wq

@@ -20,6 +20,14 @@ int cuda_status(cudaError_t e) {
   return WQ_ERR_CUDA;
 }
 
+}  // namespace
+
+namespace wq {
+int note_cuda_error(cudaError_t e) { return cuda_status(e); }
+}  // namespace wq
+
+namespace {
+
 // The kernels are built for sm_100a only: refuse any other device up front instead of
 // failing inside a launch. Cached per device ordinal.
 int check_device() {
@@ -345,6 +353,7 @@ const char* wq_status_str(int status) {
     case WQ_ERR_ALIGN: return "WQ_ERR_ALIGN: pointer not aligned as required";
     case WQ_ERR_CUDA: return "WQ_ERR_CUDA: a CUDA call or launch failed";
     case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+    case WQ_ERR_SCRATCH: return "WQ_ERR_SCRATCH: the launch needs more scratch than the library's static array holds";
     default: return "unknown wq_status";
   }
 }

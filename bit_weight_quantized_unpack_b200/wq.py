@@ -22,7 +22,8 @@ _lib = ctypes.CDLL(_LIB_PATH)
 
 WQ_INT4, WQ_INT2, WQ_TERNARY = 0, 1, 2
 FMT = {"int4": WQ_INT4, "int2": WQ_INT2, "ternary": WQ_TERNARY}
-WQ_OK, WQ_ERR_ARG, WQ_ERR_SHAPE, WQ_ERR_ALIGN, WQ_ERR_CUDA, WQ_ERR_UNSUPPORTED = range(6)
+WQ_OK, WQ_ERR_ARG, WQ_ERR_SHAPE, WQ_ERR_ALIGN, WQ_ERR_CUDA, WQ_ERR_UNSUPPORTED, WQ_ERR_SCRATCH = range(7)
+WQ_ARGMAX_STATIC_SCRATCH_BYTES = 16384
 WQ_LINEAR_SET_MAX = 256
 
 _i64, _p, _i = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
@@ -45,6 +46,7 @@ _sig = {
     "wq_device_errors": (_i, [ctypes.POINTER(ctypes.c_uint), _i, _p]),
     "wq_argmax_workspace_bytes": (ctypes.c_size_t, []),
     "wq_gemv_argmax": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p, _p, ctypes.c_size_t, _p]),
+    "wq_gemv_argmax_static": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p, _p]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -118,6 +120,13 @@ def wq_gemv_argmax(x, codes, scale, zero, fmt, N, K, y, argmax, workspace, works
     _check(_lib.wq_gemv_argmax(_ptr(x), _ptr(codes), _ptr(scale), _ptr(zero), _fmt(fmt), N, K,
                                _ptr(y), _ptr(argmax), _ptr(workspace), workspace_bytes,
                                _stream(stream)), "wq_gemv_argmax")
+
+
+def wq_gemv_argmax_static(x, codes, scale, zero, fmt, N, K, y, argmax, stream=None) -> None:
+    """wq_gemv_argmax using the library's own static scratch (no work space argument)."""
+    _check(_lib.wq_gemv_argmax_static(_ptr(x), _ptr(codes), _ptr(scale), _ptr(zero), _fmt(fmt),
+                                      N, K, _ptr(y), _ptr(argmax), _stream(stream)),
+           "wq_gemv_argmax_static")
 
 
 def make_linear_set(entries) -> ctypes.Array:

@@ -69,7 +69,8 @@ typedef enum {
   WQ_ERR_SHAPE = 2,        /* N, K or M outside the supported range, K % 128 != 0 */
   WQ_ERR_ALIGN = 3,        /* a pointer is not aligned as required above */
   WQ_ERR_CUDA = 4,         /* a CUDA call or launch failed (see wq_last_cuda_error) */
-  WQ_ERR_UNSUPPORTED = 5   /* valid request this build cannot serve (e.g. no sm_100 GPU) */
+  WQ_ERR_UNSUPPORTED = 5,  /* valid request this build cannot serve (e.g. no sm_100 GPU) */
+  WQ_ERR_SCRATCH = 6       /* needs more scratch than the library's static array holds */
 } wq_status;
 
 /* Bytes of packed codes for an [N, K] weight in format fmt (0 on invalid arguments):
@@ -149,6 +150,26 @@ size_t wq_argmax_workspace_bytes(void);
 int wq_gemv_argmax(const uint16_t* x, const void* codes, const uint16_t* scale,
                    const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* y,
                    int32_t* argmax, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of the library's own device array that wq_gemv_argmax_static uses as its scratch. */
+#define WQ_ARGMAX_STATIC_SCRATCH_BYTES 16384
+
+/* wq_gemv_argmax for callers that cannot give the library a work space: an engine that owns
+ * all device memory through its own pool and does not let libraries call cudaMalloc, or a
+ * decode loop in which an allocation (which can synchronise the device) is not acceptable.
+ * There is no counterpart on the pages; this is a deployment convenience.
+ * Same arguments and results as wq_gemv_argmax, without workspace / workspace_bytes. The
+ * scratch is a static array of WQ_ARGMAX_STATIC_SCRATCH_BYTES bytes inside libwq, held by
+ * every GPU that loads the library until the process exits; the call allocates nothing.
+ * It returns WQ_ERR_SCRATCH, before any launch, if its launch on the current device would
+ * need more (16 + 8 bytes per CTA, i.e. more than 2046 CTAs).
+ * The first call on a device looks up the array's address on that device (make that first
+ * call before any stream capture). Each call clears the array's header on `stream` before
+ * its kernel runs. All calls share the one array: two calls whose work overlaps on the GPU
+ * (different streams, not ordered by events) race and may return a wrong row. */
+int wq_gemv_argmax_static(const uint16_t* x, const void* codes, const uint16_t* scale,
+                          const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* y,
+                          int32_t* argmax, void* stream);
 
 /* Static string naming a status code. */
 const char* wq_status_str(int status);
