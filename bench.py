@@ -237,7 +237,27 @@ def bench_rows(args, pk):
         del copies
         torch.cuda.empty_cache()
     rows.update(bench_batch_sweep(args, pk))
+    rows.update(bench_7b_set(args, pk))
     return rows
+
+
+def bench_7b_set(args, pk):
+    """One decoded token of the Qwen2.5-7B-shaped set (197 int4 matrices, 3.76 GB) in one
+    wq_linear_set call; larger than L2 by itself, so one copy suffices."""
+    sets, weights, _, _ = build_set(3, copies=1)
+    nbytes = weights * INT4_BYTES_PER_WEIGHT
+    s = sets[0]
+    from bit_weight_quantized_unpack_b200 import wq
+
+    def step(i):
+        wq.wq_linear_set(s["desc"], s["count"], "int4")
+    ms = time_steps(step, 20 if not args.quick else 5, 3, 1)
+    out = {"gemv_set_qwen7b_int4": {"ms": ms, "GBps": nbytes / ms / 1e6,
+                                    "frac_hbm": nbytes / ms / 1e6 / pk["hbm_gbs"],
+                                    "implied_tok_s": 1e3 / ms}}
+    del sets, s
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 64, 512, 2048)):
