@@ -42,25 +42,30 @@ namespace {
 
 constexpr int W = kStreamWarps;
 constexpr int T = 32 * W;
-constexpr int SLOT_CODES = kStreamSlotCodes;
-constexpr int XU = 17;  // staged activation units (16 bytes) per 128-weight group
+constexpr int TERN = 1;  // format tag of ternary (5 trits per byte, 26 bytes per group)
 
 // Chunk permutation of group g (XOR mask on the chunk index), shared by the codes reads and
 // the staged activation layout.
 template <int BITS>
 __host__ __device__ __forceinline__ int xrot(int g) {
-  return BITS == 4 ? (g >> 1) & 3 : (g >> 2) & 1;
+  return BITS == 4 ? (g >> 1) & 3 : BITS == 2 ? (g >> 2) & 1 : 0;
 }
 
+// Per format (BITS = 4, 2, or TERN): bytes of codes per cell (one group), ring slot layout
+// (codes, then scales, then zeros for the integer formats), staged activation units per group.
 template <int BITS>
 struct Fmt {
-  static constexpr int CB = 128 * BITS / 8;    // codes bytes per cell (one group): 64 / 32
-  static constexpr int CH = CB / 16;           // 16-byte chunks per cell: 4 / 2
-  static constexpr int UPC = 16 / CH;          // activation units per chunk: 4 / 8
-  static constexpr int SPS = SLOT_CODES / (32 * CB);  // steps of 32 cells per ring slot: 2 / 4
-  static constexpr int GPSL = SLOT_CODES / CB;        // groups per ring slot: 64 / 128
-  static constexpr int META = 2 * GPSL;               // bytes of scales (and of zeros) per slot
-  static constexpr int SLOT = SLOT_CODES + 2 * META;
+  static constexpr bool TRN = BITS == TERN;
+  static constexpr int CB = TRN ? 26 : 128 * BITS / 8;  // codes bytes per cell: 64 / 32 / 26
+  static constexpr int CH = TRN ? 1 : CB / 16;          // 16-byte chunks per cell: 4 / 2
+  static constexpr int UPC = 16 / CH;                   // activation units per chunk: 4 / 8
+  static constexpr int SPS = TRN ? 4 : kStreamSlotCodes / (32 * CB);  // steps of 32 cells per slot
+  static constexpr int SC = 32 * SPS * CB;              // codes bytes per slot: 4096 / 4096 / 3328
+  static constexpr int GPSL = 32 * SPS;                 // groups per ring slot: 64 / 128 / 128
+  static constexpr int META = 2 * GPSL;                 // bytes of scales (and of zeros) per slot
+  static constexpr int SLOT = SC + (TRN ? 1 : 2) * META;
+  static constexpr int XU = TRN ? 27 : 17;              // staged activation units per group
+  static constexpr int LUT = TRN ? 256 * 4 : 0;         // byte -> five base-3 digits (shared memory)
 };
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
@@ -167,6 +172,46 @@ __device__ __forceinline__ void cell_dot(uint32_t cell, uint32_t xg, uint32_t xs
   }
 }
 
+// Ternary: out[m] = 2^-24 * sum_k x_mk t_k over one cell (26 bytes at the 2-byte aligned
+// shared address `cell`). lut: shared table of 256 words, word b = the base-3 digits
+// d_i = t_i + 1 of byte b at bits 0, 16 (d0, d1), 2, 18 (d2, d3) and 4 (d4) (digits 1,
+// i.e. zero trits, for the invalid bytes 243..255). Masking two digits gives the binary16
+// subnormals d 2^-24; one packed subtract of 2^-24 gives (d - 1) 2^-24 = t 2^-24 exactly.
+// xg: the group's 26 staged activation units of row 0 (unit j = x[5j .. 5j + 4]), rows xs
+// bytes apart. Each product is exact in binary32.
+template <int MT>
+__device__ __forceinline__ void cell_dot_ternary(uint32_t cell, uint32_t xg, uint32_t xs, uint32_t lut,
+                                                 float (&out)[MT]) {
+  float a[MT][2];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) a[m][0] = a[m][1] = 0.f;
+#pragma unroll
+  for (int h = 0; h < 13; ++h) {
+    const uint32_t two = lds16(cell + 2 * h);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = 2 * h + e;
+      uint32_t w;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(lut + 4 * ((two >> (8 * e)) & 0xFFu)));
+      const uint32_t t01 = hsub2_u32(w & 0x00030003u, 0x00010001u);         // t0, t1
+      const uint32_t t23 = hsub2_u32((w >> 2) & 0x00030003u, 0x00010001u);  // t2, t3
+      const uint32_t t4 = hsub2_u32((w >> 4) & 0x00000003u, 0x00010001u);   // t4 (low half)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint4 xw = lds128(xg + m * xs + 16 * j);
+        float& A = a[m][e];
+        A = fma_f16f16_f32(lo16(t01), lo16(xw.x), A);
+        A = fma_f16f16_f32(hi16(t01), hi16(xw.x), A);
+        A = fma_f16f16_f32(lo16(t23), lo16(xw.y), A);
+        A = fma_f16f16_f32(hi16(t23), hi16(xw.y), A);
+        A = fma_f16f16_f32(lo16(t4), lo16(xw.z), A);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) out[m] = a[m][0] + a[m][1];
+}
+
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -211,8 +256,8 @@ __device__ __forceinline__ Seg warp_seg(const StreamMat& M, int b0, int b1, int 
   const int wb1 = b0 + (int)((int64_t)(b1 - b0) * (w + 1) / W);
   const int64_t r0 = (int64_t)wb0 * M.RA;
   const int64_t r1 = (int64_t)wb1 * M.RA < M.N ? (int64_t)wb1 * M.RA : M.N;
-  const int64_t rb = (int64_t)M.K * BITS / 8;
   const int G = M.K / kGroup;
+  const int64_t rb = (int64_t)G * Fmt<BITS>::CB;
   Seg s;
   s.rows = r1 > r0 ? (int)(r1 - r0) : 0;
   s.row0 = (int)r0;
@@ -240,7 +285,7 @@ struct Prod {
 // AM: also keep this lane's best (fp16 value, row) among the rows it completes, for the fused
 // argmax (ties to the lowest row).
 template <int BITS, int MT, bool AM, class Issue>
-__device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint32_t ring,
+__device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint32_t lut, uint32_t ring,
                                         uint32_t bars, int slots, int& cslot, uint32_t& cphase, int& consumed,
                                         bool& dead, Issue& issue, int lane, float& bv, int& bi) {
   using F = Fmt<BITS>;
@@ -252,17 +297,23 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
   // the matrix's last partial 16-byte unit of scales / zeros, if this segment ends there:
   // loaded now, stored into its ring slot before that slot is read
   const int rem = ncells & 7;
+  // ternary rows are 26 K / 128 bytes: a segment at the end of a matrix may end inside a
+  // 16-byte unit; those last bytes are loaded here too
+  const int crem = F::TRN ? (int)(seg.bytes & 15) : 0;
+  uint32_t cr = 0;
+  if (F::TRN && crem && lane >= 16 && lane < 16 + crem)
+    cr = __ldg(seg.codes + (seg.bytes & ~(int64_t)15) + (lane - 16));
   uint16_t rs = 0, rz = 0;
   if (rem) {
     const int gb = ncells - rem;
     if (lane < rem) rs = ld_u16(seg.s + gb + lane);
-    if (lane >= 8 && lane < 8 + rem) rz = ld_u16(seg.z + gb + lane - 8);
+    if (!F::TRN && lane >= 8 && lane < 8 + rem) rz = ld_u16(seg.z + gb + lane - 8);
   }
   // group gp of row `row` of the segment: this lane's cell
   const uint32_t gmul = ((1u << 20) + G - 1) / G;  // floor(n / G) = (n * gmul) >> 20 for n < G + 32, G < 32
   int row = G >= 32 ? 0 : (int)(((uint32_t)lane * gmul) >> 20);
   int gp = lane - row * G;
-  const uint32_t xs = (uint32_t)(G * XU * 16);  // bytes between the staged rows of X
+  const uint32_t xs = (uint32_t)(G * F::XU * 16);  // bytes between the staged rows of X
   float carry[MT];  // per row of X: part of the row of W that continues from the previous step
 #pragma unroll
   for (int m = 0; m < MT; ++m) carry[m] = 0.f;
@@ -272,15 +323,22 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
       const bool ok = tc::mbar_wait(bars + 8 * cslot, cphase);
       if (!__all_sync(0xffffffffu, ok)) dead = true;
     }
+    if (F::TRN && crem && k == nslots - 1) {
+      const int cl = (int)(seg.bytes & ~(int64_t)15) - k * F::SC;  // slot offset of the tail
+      if (lane >= 16 && lane < 16 + crem)
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(slot + cl + lane - 16), "r"(cr));
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+    }
     if (rem && k == nslots - 1) {
       const int gl = ncells - rem - k * F::GPSL;
-      if (lane < rem) asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + SLOT_CODES + 2 * (gl + lane)), "h"(rs));
-      if (lane >= 8 && lane < 8 + rem)
-        asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + SLOT_CODES + F::META + 2 * (gl + lane - 8)), "h"(rz));
+      if (lane < rem) asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + F::SC + 2 * (gl + lane)), "h"(rs));
+      if (!F::TRN && lane >= 8 && lane < 8 + rem)
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + F::SC + F::META + 2 * (gl + lane - 8)), "h"(rz));
       tc::fence_proxy_async_smem();  // the slot is refilled by bulk copies later
       __syncwarp();
     }
-    const uint32_t cell0 = slot + lane * F::CB, meta0 = slot + SLOT_CODES + 2 * lane;
+    const uint32_t cell0 = slot + lane * F::CB, meta0 = slot + F::SC + 2 * lane;
 #pragma unroll
     for (int ss = 0; ss < F::SPS; ++ss) {
       const int st = k * F::SPS + ss;
@@ -290,7 +348,14 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
 #pragma unroll
       for (int m = 0; m < MT; ++m) v[m] = 0.f;
       if (valid && !dead) {
-        const uint16_t sb = lds16(meta0 + 64 * ss), zb = lds16(meta0 + 64 * ss + F::META);
+        const uint16_t sb = lds16(meta0 + 64 * ss);
+        if constexpr (F::TRN) {
+          cell_dot_ternary<MT>(cell0 + 32 * F::CB * ss, xb + 16 * F::XU * gp, xs, lut, v);
+          const float sf = __half2float(__ushort_as_half(sb)) * 16777216.f;  // 2^24 back, exactly
+#pragma unroll
+          for (int m = 0; m < MT; ++m) v[m] *= sf;
+        } else {
+        const uint16_t zb = lds16(meta0 + 64 * ss + F::META);
         // chunks in an order permuted by the group index, so that the lanes of one
         // shared-memory phase (consecutive cells) hit different bank groups; the staged
         // activations of each group are stored in that same order (see stage_x), so the
@@ -304,10 +369,11 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
           ox[c] = 16 * F::UPC * c;
         }
         // the cell's sum carries a factor 2^-24; the scale times 2^24 takes it back (exactly)
-        cell_dot<BITS, MT>(cell0 + 32 * F::CB * ss, xb + 16 * XU * gp, xs, oc, ox, zb, v);
+        cell_dot<BITS, MT>(cell0 + 32 * F::CB * ss, xb + 16 * F::XU * gp, xs, oc, ox, zb, v);
         const float s24 = __half2float(__ushort_as_half(sb)) * 16777216.f;
 #pragma unroll
         for (int m = 0; m < MT; ++m) v[m] *= s24;
+        }
       }
       // segmented inclusive scan over the lanes of each row within this step
       const int lim = gp < lane ? gp : lane;
@@ -379,6 +445,18 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
   const uint32_t ring = sbase + w * slots * F::SLOT;
   const uint32_t bars = sbase + W * slots * F::SLOT + 8 * w * slots;
   const uint32_t xbase = sbase + W * slots * (F::SLOT + 8);
+  const uint32_t lut = xbase + P.xbufs * P.xbuf_bytes;  // ternary byte -> trits table
+  if constexpr (F::TRN) {
+    for (int e = threadIdx.x; e < 256; e += T) {
+      uint32_t d[5] = {1, 1, 1, 1, 1};  // digit 1 = trit 0 (also for the invalid bytes)
+      if (e < 243) {
+        int b = e;
+        for (int i = 0; i < 5; ++i, b /= 3) d[i] = (uint32_t)(b % 3);
+      }
+      const uint32_t word = d[0] | d[1] << 16 | d[2] << 2 | d[3] << 18 | d[4] << 4;
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(lut + 4 * e), "r"(word) : "memory");
+    }
+  }
 
   const int64_t share = (P.total_cost + gridDim.x - 1) / gridDim.x;
   const int64_t lo = share * blockIdx.x, hi = lo + share;
@@ -416,17 +494,20 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
       pd.gleft = sg.groups;
     }
     const uint32_t bar = bars + 8 * slot, dst = ring + slot * F::SLOT;
-    int cb = SLOT_CODES, gc = F::GPSL;
-    if (pd.cleft < SLOT_CODES) {
+    int cb = F::SC, gc = F::GPSL;
+    if (pd.cleft < F::SC) {
       cb = pd.cleft;
       gc = pd.gleft;
     }
-    const uint32_t mb = 2u * (uint32_t)(gc & ~7);  // whole 16-byte units; the rest is done by the consumer
-    if (lane == 0) tc::mbar_arrive_expect_tx(bar, (uint32_t)cb + 2 * mb);
-    if (lane == 0 || (lane < 3 && mb)) {
+    // whole 16-byte units of scales / zeros (and, for ternary, of codes); the rest, at the
+    // end of a matrix, is loaded by the consumer lanes
+    const uint32_t mb = 2u * (uint32_t)(gc & ~7);
+    const uint32_t cbb = (uint32_t)cb & ~15u;
+    if (lane == 0) tc::mbar_arrive_expect_tx(bar, cbb + (F::TRN ? 1 : 2) * mb);
+    if (lane == 0 || (lane < (F::TRN ? 2 : 3) && mb)) {
       const void* src = lane == 0 ? (const void*)pd.c : lane == 1 ? (const void*)pd.s : (const void*)pd.z;
-      const uint32_t d = lane == 0 ? dst : dst + SLOT_CODES + (lane - 1) * F::META;
-      bulk_g2s(d, src, lane == 0 ? (uint32_t)cb : mb, bar);
+      const uint32_t d = lane == 0 ? dst : dst + F::SC + (lane - 1) * F::META;
+      bulk_g2s(d, src, lane == 0 ? cbb : mb, bar);
     }
     pd.c += cb;
     pd.s += gc;
@@ -460,11 +541,27 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
   // 17 g .. 17 g + 15 of the row, its chunks (UPC units each) in the order of the group's
   // chunk permutation
   auto stage_x = [&](const StreamMat& M, uint32_t xb) {
-    const int units = M.K / 8, rowu = (M.K / kGroup) * XU;
+    if constexpr (F::TRN) {
+      // ternary: unit j of group g holds x[128 g + 5 j .. + 4] (three values in unit 25);
+      // 10-byte pieces, so plain loads and stores (made visible by the caller's barrier)
+      const int G = M.K / kGroup, per = G * 26;
+      for (int t = threadIdx.x; t < MT * per; t += T) {
+        const int m = t / per, r = t - m * per, g = r / 26, j = r - g * 26;
+        const uint16_t* src = M.x + (size_t)m * M.K + kGroup * g + 5 * j;
+        uint32_t h[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) h[i] = (5 * j + i < kGroup) ? (uint32_t)__ldg(src + i) : 0u;
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(xb + 16 * (m * G * F::XU + F::XU * g + j)),
+                     "r"(h[0] | h[1] << 16), "r"(h[2] | h[3] << 16), "r"(h[4]), "r"(0u)
+                     : "memory");
+      }
+      return;
+    }
+    const int units = M.K / 8, rowu = (M.K / kGroup) * F::XU;
     for (int t = threadIdx.x; t < MT * units; t += T) {
       const int m = t / units, u = t - m * units;
       const int g = u >> 4, lc = (u & 15) / F::UPC, i = u & (F::UPC - 1);
-      const int pu = m * rowu + XU * g + F::UPC * (lc ^ xrot<BITS>(g)) + i;
+      const int pu = m * rowu + F::XU * g + F::UPC * (lc ^ xrot<BITS>(g)) + i;
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + 16 * pu), "l"(M.x + (size_t)8 * t)
                    : "memory");
     }
@@ -500,7 +597,8 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     cta_units(M, lo, hi, b0, b1);
     const Seg seg = warp_seg<BITS>(M, b0, b1, w);
     if (seg.rows > 0)
-      consume<BITS, MT, AM>(seg, M, xb, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane, am_v, am_i);
+      consume<BITS, MT, AM>(seg, M, xb, lut, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane, am_v,
+                            am_i);
   }
 
   // ---- fused argmax: warp, CTA, then the last CTA to finish combines every CTA's partial
@@ -584,7 +682,7 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
     // rows per unit: segments start at multiples of RA rows, so that their scales and zeros
     // start on a 16-byte boundary (8 groups)
     const int RA = 8 / gcd_int(G, 8);
-    const int64_t row_cost = (int64_t)K * BITS / 8 + 4 * G;
+    const int64_t row_cost = (int64_t)G * F::CB + (F::TRN ? 2 : 4) * G;
     StreamMat& m = p.m[i];
     m.codes = d[i].codes;
     m.scale = d[i].scale;
@@ -606,12 +704,12 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   p.total_cost = cost;
   p.am_ws = nullptr;
   p.am_out = nullptr;
-  p.xbuf_bytes = (mt * (max_k / kGroup) * XU * 16 + 127) & ~127;
+  p.xbuf_bytes = (mt * (max_k / kGroup) * F::XU * 16 + 127) & ~127;
   p.errors = device_error_word();
   if (!p.errors) return 0;
   // two ring slots per warp; two activation buffers when four CTAs still fit on an SM
   // (measured best on the 0.5B decode set), else one; then as many CTAs as fit
-  const int ring = W * 2 * (F::SLOT + 8);
+  const int ring = W * 2 * (F::SLOT + 8) + F::LUT;
   const int two = ring + 2 * p.xbuf_bytes, one = ring + p.xbuf_bytes;
   const int bytes = (kStreamSmPool / (two + 1024) >= kStreamMaxCtasPerSm) ? two : one;
   if (bytes > kStreamMaxSmem) return 0;
@@ -683,11 +781,12 @@ cudaError_t launch_b(const StreamParams& p, int mt, int smem, cudaStream_t strea
 
 int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int mt) {
   if (count < 1 || count > kStreamMaxMats || mt < 1 || mt > kStreamMaxRows) return 0;
-  return bits == 4 ? plan_t<4>(p, count, d, mt) : plan_t<2>(p, count, d, mt);
+  return bits == 4 ? plan_t<4>(p, count, d, mt) : bits == 2 ? plan_t<2>(p, count, d, mt) : plan_t<TERN>(p, count, d, mt);
 }
 
 cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem, cudaStream_t stream) {
-  return bits == 4 ? launch_b<4>(p, mt, smem, stream) : launch_b<2>(p, mt, smem, stream);
+  return bits == 4 ? launch_b<4>(p, mt, smem, stream)
+                   : bits == 2 ? launch_b<2>(p, mt, smem, stream) : launch_b<TERN>(p, mt, smem, stream);
 }
 
 cudaError_t launch_gemv_stream_argmax(const StreamParams& p, int bits, int smem, cudaStream_t stream) {

@@ -58,7 +58,7 @@ struct StreamDesc {
   int64_t N, K;
 };
 
-// Fills p for a set of `count` matrices of one format (bits 4 or 2), each multiplied by mt
+// Fills p for a set of `count` matrices of one format (bits 4, 2, or 1 for ternary), each multiplied by mt
 // rows of X (X [mt, K] and Y [mt, N] row-major), and returns the bytes of dynamic shared
 // memory a CTA needs, or 0 if this kernel cannot serve the set (pointers not 16-byte
 // aligned, or activations too long to stage).

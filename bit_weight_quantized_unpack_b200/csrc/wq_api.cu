@@ -117,11 +117,11 @@ bool plan_bulk(wq::BulkParams& p, int fmt, int count, const wq_linear_desc* d) {
 // memory.
 int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStream_t stream, bool* done) {
   *done = false;
-  if (fmt == WQ_TERNARY || count > wq::kStreamMaxMats || M > wq::kStreamMaxRows) return WQ_OK;
+  if (count > wq::kStreamMaxMats || M > wq::kStreamMaxRows) return WQ_OK;
   static thread_local wq::StreamParams sp;
   static thread_local wq::StreamDesc sd[wq::kStreamMaxMats];
   for (int i = 0; i < count; ++i) sd[i] = {d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K};
-  const int bits = fmt == WQ_INT4 ? 4 : 2;
+  const int bits = fmt == WQ_INT4 ? 4 : fmt == WQ_INT2 ? 2 : 1;  // 1: ternary
   const int smem = wq::stream_plan(sp, bits, count, sd, (int)M);
   if (smem == 0) return WQ_OK;
   *done = true;
