@@ -56,8 +56,12 @@ __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
   return d;
 }
 
+// (v & mask) | orv as one three-input logic op (truth table 0xEA = (a & b) | c); written out
+// because the plain C expression with two constant operands measured as two instructions.
 __device__ __forceinline__ uint32_t lop_and_or(uint32_t v, uint32_t mask, uint32_t orv) {
-  return (v & mask) | orv;  // one LOP3
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(v), "r"(mask), "r"(orv));
+  return d;
 }
 
 }  // namespace wq
