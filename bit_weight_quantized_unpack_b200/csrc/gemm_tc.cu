@@ -49,7 +49,11 @@ constexpr int XSTAGES = WQ_TC_XSTAGES;  // activation tiles [bn x 64] (read from
 constexpr int CRING = WQ_TC_CRING;      // codes ring slots: CRING - 1 of a team's k-blocks in flight
 constexpr int ASTAGES = WQ_TC_ASTAGES;  // dequantised weight tiles (written by CUDA cores, read by MMA)
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB of dequantised fp16 weights
-constexpr int B_BYTES = kTcMaxBN * BK * 2;      // 32 KB of activations
+#ifndef WQ_TC_XBN
+#define WQ_TC_XBN kTcMaxBN
+#endif
+constexpr int XBN = WQ_TC_XBN;                  // tokens one activation stage holds
+constexpr int B_BYTES = XBN * BK * 2;           // activations of one stage
 constexpr int CSLOT_BYTES = 2 * BM * BK / 2;   // one ring slot: 32 B of codes for each of 256 threads
 constexpr int OFF_A = 0;
 constexpr int OFF_X = OFF_A + ASTAGES * A_BYTES;
@@ -458,7 +462,7 @@ bool tc_plan_mat(TcMat& t, const uint16_t* X, int M, const void* codes, const ui
 
 int tc_bn_for(int M) {
   const int bn = ((M + 15) / 16) * 16;
-  return bn < kTcMaxBN ? bn : kTcMaxBN;
+  return bn < XBN ? bn : XBN;
 }
 
 template <int CAP>

@@ -3,6 +3,7 @@
 #include <limits.h>
 #include <string.h>
 
+#include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_bulk.cuh"
@@ -128,6 +129,20 @@ int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStrea
   return cuda_status(wq::launch_gemv_stream(sp, bits, (int)M, smem, stream));
 }
 
+// Skinny-batch GEMM for an int4 set with kSkMinM <= M <= kSkMaxM: needs 16-byte aligned
+// codes and activations.
+int try_skinny(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStream_t stream, bool* done) {
+  *done = false;
+  if (fmt != WQ_INT4 || count > wq::kSkMaxMats || M < wq::kSkMinM || M > wq::kSkMaxM) return WQ_OK;
+  static thread_local wq::SkParams kp;
+  static thread_local wq::SkDesc kd[wq::kSkMaxMats];
+  for (int i = 0; i < count; ++i) kd[i] = {d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K};
+  const int smem = wq::skinny_plan(kp, count, kd, (int)M);
+  if (smem == 0) return WQ_OK;
+  *done = true;
+  return cuda_status(wq::launch_gemm_skinny(kp, smem, stream));
+}
+
 // Row-per-lane kernel for a batch-1 set (int4 / int2): needs 32-byte aligned codes
 // (its loads are whole 32-byte sectors) and K small enough to stage x in shared memory.
 int try_rows(int fmt, int count, const wq_linear_desc* d, cudaStream_t stream, bool* done) {
@@ -181,6 +196,12 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
   if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
   if (!aligned(X, 16) || !aligned(Y, 2)) return WQ_ERR_ALIGN;
   if ((st = check_device()) != WQ_OK) return st;
+  {
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, M};
+    bool done = false;
+    const int r = try_skinny(fmt, 1, &d, M, (cudaStream_t)stream, &done);
+    if (done) return r;
+  }
   if (fmt == WQ_INT4 && M >= wq::kTcMinM) {
     // tensor-core path: 128-row weight tiles x up to 256 tokens
     static thread_local wq::TcParams tp;  // ~20 KB: kept off the stack, one per thread
@@ -249,6 +270,11 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   }
   int st0 = check_device();
   if (st0 != WQ_OK) return st0;
+  {
+    bool done = false;
+    const int r = try_skinny(fmt, count, descs, M, (cudaStream_t)stream, &done);
+    if (done) return r;
+  }
   if (fmt == WQ_INT4 && M >= wq::kTcMinM) {
     // tensor-core GEMM: persistent launches of up to kTcMaxMats matrices each
     static thread_local wq::TcParams tp;
