@@ -43,15 +43,7 @@ namespace wq {
 
 namespace {
 
-constexpr int kThreads = 32 * kSkWarps;
 
-__device__ __forceinline__ uint4 ld_codes16(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
@@ -90,16 +82,84 @@ __device__ __forceinline__ uint32_t neg_zc(uint16_t zb) {
 // stride of 16 (mod 128) bytes.
 __device__ __forceinline__ uint32_t xchunk_off(uint32_t c) { return (c ^ (((c >> 3) & 1u) << 1)) << 4; }
 
-struct Item {
-  int unit, ch, mi;
+__device__ __forceinline__ void cp_async16_l2(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// wait until at most n (0 <= n < kSkRing) of this thread's newest copy groups are pending
+__device__ __forceinline__ void cp_async_wait_upto(int n) {
+  static_assert(kSkRing == 4, "one case per ring depth");
+  if (n <= 0) cp_async_wait<0>();
+  else if (n == 1) cp_async_wait<1>();
+  else if (n == 2) cp_async_wait<2>();
+  else cp_async_wait<3>();
+}
+
+// d = A * B with a zero accumulator (first MMA of a group)
+__device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// A position in a CTA's work: item = window [ws, we) of slabs (one per warp) of matrix mi and
+// activation chunk ch (groups g0 .. g0 + ng - 1); step gl = group g0 + gl of the item.
+struct Walk {
+  int ws, we, mi, ch, g0, ng, gl;
 };
 
 template <int CAP>
-__device__ __forceinline__ int find_mat(const SkParamsT<CAP>& P, int unit) {
+__device__ __forceinline__ void item_fill(const SkParamsT<CAP>& P, Walk& w, int hi) {
+  const SkMat& m = P.m[w.mi];
+  w.we = min(min(w.ws + kSkWarps, m.slab_end), hi);
+  w.g0 = w.ch * m.kc;
+  w.ng = min(m.kc, m.G - w.g0);
+}
+
+// the next item (ch + 1, or the next window); false past the CTA's last slab
+template <int CAP>
+__device__ __forceinline__ bool item_next(const SkParamsT<CAP>& P, Walk& w, int hi) {
+  if (w.ch + 1 < P.m[w.mi].nch) {
+    ++w.ch;
+  } else {
+    w.ws = w.we;
+    if (w.ws >= hi) return false;
+    while (w.ws >= P.m[w.mi].slab_end) ++w.mi;
+    w.ch = 0;
+  }
+  item_fill(P, w, hi);
+  return true;
+}
+
+// first slab whose cost position is >= c (slab j of matrix i sits at cost_begin_i + j G_i)
+template <int CAP>
+__device__ __forceinline__ int slab_at(const SkParamsT<CAP>& P, int64_t c) {
+  if (c >= P.total_cost) return P.total_slabs;
   int lo = 0, hi = P.count - 1;
-  while (lo < hi) {  // last matrix whose unit_begin <= unit
+  while (lo < hi) {  // last matrix with cost_begin <= c
     const int mid = (lo + hi + 1) >> 1;
-    if (P.m[mid].unit_begin <= unit) lo = mid; else hi = mid - 1;
+    if (P.m[mid].cost_begin <= c) lo = mid; else hi = mid - 1;
+  }
+  const SkMat& m = P.m[lo];
+  return m.slab_begin + (int)((c - m.cost_begin + m.G - 1) / m.G);
+}
+
+template <int CAP>
+__device__ __forceinline__ int mat_of_slab(const SkParamsT<CAP>& P, int s) {
+  int lo = 0, hi = P.count - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.m[mid].slab_begin <= s) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -107,140 +167,220 @@ __device__ __forceinline__ int find_mat(const SkParamsT<CAP>& P, int unit) {
 }  // namespace
 
 template <int TB, int CAP>
-__global__ void __launch_bounds__(kThreads, kSkCtasPerSm) gemm_skinny_kernel(const __grid_constant__ SkParamsT<CAP> P) {
+__global__ void __launch_bounds__(kSkThreads, 1) gemm_skinny_kernel(const __grid_constant__ SkParamsT<CAP> P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int M = P.M;
-  constexpr int NT = 8 * TB;                       // staged token rows (zero past M)
-  constexpr int TPT = kThreads / NT;               // staging threads per token row
-  const int stage_n = threadIdx.x / TPT, stage_c0 = threadIdx.x % TPT;
+  constexpr int NT = 8 * TB;                  // staged token rows (rows past M are never read
+  constexpr int TPT = kSkThreads / NT;        // into a stored output)
+  const int stage_n = tid / TPT, stage_c0 = tid % TPT;
+  constexpr uint32_t kSlot = 2u * kSkThreads * 16u;   // ring slot: [row g | row g + 8][thread][16 B]
+  const uint32_t ring_me = sbase + 2u * (uint32_t)P.buf_bytes + 16u * (uint32_t)tid;
 
-  // stage the activations of item it into buffer b (cp.async; rows past M are zeroed)
-  auto stage = [&](const Item& it, int b) {
-    const SkMat& Mt = P.m[it.mi];
-    const int G = Mt.K / kGroup;
-    const int g0 = it.ch * Mt.kc, ng = min(Mt.kc, G - g0);
-    const uint32_t ts = (uint32_t)Mt.kc * 256u + 16u;
-    const uint32_t row = sbase + (uint32_t)b * (uint32_t)P.buf_bytes + (uint32_t)stage_n * ts;
-    const int nc = 16 * ng;
+  // this CTA's slabs: a contiguous range of about equal cost
+  const int64_t C = P.total_cost;
+  const int lo = slab_at(P, C * blockIdx.x / gridDim.x);
+  const int hi = slab_at(P, C * (blockIdx.x + 1) / gridDim.x);
+  if (lo >= hi) return;
+
+  auto stage_x = [&](const Walk& it, int b) {
     if (stage_n < M) {
-      const uint16_t* src = Mt.x + (size_t)stage_n * Mt.K + (size_t)g0 * kGroup;
-      for (int c = stage_c0; c < nc; c += TPT) cp_async16(row + xchunk_off((uint32_t)c), src + 8 * c);
-    } else {
-      for (int c = stage_c0; c < nc; c += TPT)
-        asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(row + xchunk_off((uint32_t)c)), "r"(0u) : "memory");
+      const SkMat& m = P.m[it.mi];
+      const uint32_t row = sbase + (uint32_t)b * (uint32_t)P.buf_bytes + (uint32_t)stage_n * ((uint32_t)m.kc * 256u + 16u);
+      const uint16_t* src = m.x + (size_t)stage_n * m.K + (size_t)it.g0 * kGroup;
+      for (int c = stage_c0; c < 16 * it.ng; c += TPT) cp_async16(row + xchunk_off((uint32_t)c), src + 8 * c);
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  auto next_item = [&](Item it) {
-    if (it.ch + 1 < P.m[it.mi].nch) {
-      ++it.ch;
-    } else {
-      it.unit += gridDim.x;
-      it.ch = 0;
-      if (it.unit < P.total_units) it.mi = find_mat(P, it.unit);
-    }
-    return it;
   };
 
-  Item cur{(int)blockIdx.x, 0, 0};
-  if (cur.unit >= P.total_units) return;
-  cur.mi = find_mat(P, cur.unit);
-  stage(cur, 0);
+  Walk it;
+  it.ws = lo;
+  it.mi = mat_of_slab(P, lo);
+  it.ch = 0;
+  it.gl = 0;
+  item_fill(P, it, hi);
+  stage_x(it, 0);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // Fetch cursor (kSkRing - 1 steps ahead of the compute) and metadata cursor (one step
+  // ahead). Each keeps the sources of its next step in registers and walks them with pointer
+  // bumps; the item bookkeeping runs only when it moves to another item.
+  Walk f = it;
+  bool fv = true;
+  while (warp >= f.we - f.ws)
+    if (!item_next(P, f, hi)) { fv = false; break; }
+  Walk sc = f;
+  bool sv = fv;
+  const uint8_t* fp_lo = nullptr;
+  const uint8_t* fp_hi = nullptr;
+  const uint16_t* fm = nullptr;
+  auto fetch_item = [&]() {
+    const SkMat& m = P.m[f.mi];
+    const int r0 = (f.ws + warp - m.slab_begin) * 16 + g;
+    const int rl = min(r0, m.N - 1), rh = min(r0 + 8, m.N - 1);
+    fp_lo = m.codes + (size_t)rl * (m.K / 2) + (size_t)f.g0 * 64 + 16 * t;
+    fp_hi = m.codes + (size_t)rh * (m.K / 2) + (size_t)f.g0 * 64 + 16 * t;
+    // the metadata value this lane prefetches: t = 0, 1: scale of row g, g + 8; 2, 3: zero
+    fm = ((t & 2) ? m.zero : m.scale) + (size_t)((t & 1) ? rh : rl) * m.G + f.g0;
+  };
+  if (fv) fetch_item();
+  auto fetch = [&](uint32_t slot) {
+    cp_async16_l2(ring_me + slot * kSlot, fp_lo);
+    cp_async16_l2(ring_me + slot * kSlot + kSlot / 2, fp_hi);
+    prefetch_l2(fm);
+    if (++f.gl < f.ng) {
+      fp_lo += 64;
+      fp_hi += 64;
+      fm += 1;
+    } else {
+      f.gl = 0;
+      do {
+        if (!item_next(P, f, hi)) { fv = false; break; }
+      } while (warp >= f.we - f.ws);
+      if (fv) fetch_item();
+    }
+  };
+  uint32_t fslot = 0;
+#pragma unroll 1
+  for (int d = 0; d < kSkRing - 1; ++d) {
+    if (fv) fetch(fslot);
+    cp_async_commit();
+    fslot = fslot + 1 == kSkRing ? 0 : fslot + 1;
+  }
+
+  // metadata of the next step, in registers
+  const uint16_t* ms_lo = nullptr;
+  const uint16_t* ms_hi = nullptr;
+  const uint16_t* mz_lo = nullptr;
+  const uint16_t* mz_hi = nullptr;
+  auto meta_item = [&]() {
+    const SkMat& m = P.m[sc.mi];
+    const int r0 = (sc.ws + warp - m.slab_begin) * 16 + g;
+    const size_t il = (size_t)min(r0, m.N - 1) * m.G + sc.g0;
+    const size_t ih = (size_t)min(r0 + 8, m.N - 1) * m.G + sc.g0;
+    ms_lo = m.scale + il;
+    ms_hi = m.scale + ih;
+    mz_lo = m.zero + il;
+    mz_hi = m.zero + ih;
+  };
+  uint16_t ns_lo = 0, ns_hi = 0, nz_lo = 0, nz_hi = 0;
+  auto load_meta = [&]() {
+    ns_lo = ld_u16(ms_lo + sc.gl);
+    ns_hi = ld_u16(ms_hi + sc.gl);
+    nz_lo = ld_u16(mz_lo + sc.gl);
+    nz_hi = ld_u16(mz_hi + sc.gl);
+    if (++sc.gl == sc.ng) {
+      sc.gl = 0;
+      do {
+        if (!item_next(P, sc, hi)) { sv = false; break; }
+      } while (warp >= sc.we - sc.ws);
+      if (sv) meta_item();
+    }
+  };
+  if (sv) {
+    meta_item();
+    load_meta();
+  }
+
+  uint32_t xoff[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) xoff[w] = xchunk_off((uint32_t)(4 * t + w));
 
   float acc[TB][4];
 #pragma unroll
   for (int b = 0; b < TB; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
+  uint32_t cslot = 0;
+  int buf = 0;
 
-  for (int i = 0; cur.unit < P.total_units; ++i) {
-    const SkMat& Mt = P.m[cur.mi];
-    const int K = Mt.K, G = K / kGroup;
-    const int g0 = cur.ch * Mt.kc, ng = min(Mt.kc, G - g0);
-    const int n0 = (cur.unit - Mt.unit_begin) * kSkUnitRows + 16 * warp;
-    const int r_lo = min(n0 + g, Mt.N - 1), r_hi = min(n0 + g + 8, Mt.N - 1);
-    const uint8_t* c_lo = Mt.codes + (size_t)r_lo * (K / 2) + 16 * t;
-    const uint8_t* c_hi = Mt.codes + (size_t)r_hi * (K / 2) + 16 * t;
-    const uint16_t* s_lo = Mt.scale + (size_t)r_lo * G;
-    const uint16_t* s_hi = Mt.scale + (size_t)r_hi * G;
-    const uint16_t* z_lo = Mt.zero + (size_t)r_lo * G;
-    const uint16_t* z_hi = Mt.zero + (size_t)r_hi * G;
+  for (;;) {
+    const SkMat& m = P.m[it.mi];
+    const bool active = warp < it.we - it.ws;
+    Walk nx = it;
+    const bool has_next = item_next(P, nx, hi);
+    const bool restage = has_next && (nx.mi != it.mi || nx.ch != it.ch);
+    if (restage) stage_x(nx, buf ^ 1);  // these copies join this thread's next commit
 
-    // first group of this item: its loads fly while the CTA waits for the activations
-    uint4 nw_lo = ld_codes16(c_lo + (size_t)g0 * 64), nw_hi = ld_codes16(c_hi + (size_t)g0 * 64);
-    uint16_t ns_lo = ld_u16(s_lo + g0), ns_hi = ld_u16(s_hi + g0);
-    uint16_t nz_lo = ld_u16(z_lo + g0), nz_hi = ld_u16(z_hi + g0);
-
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();  // item i's activations are visible; every warp is done with item i - 1
-    const Item nxt = next_item(cur);
-    if (nxt.unit < P.total_units) stage(nxt, (i + 1) & 1);
-
-    const uint32_t ts = (uint32_t)Mt.kc * 256u + 16u;
-    // this lane's activation row (token g of block 0) in the buffer of item i
-    const uint8_t* xrow = smem + (size_t)(i & 1) * P.buf_bytes + (size_t)g * ts;
-    for (int gl = 0; gl < ng; ++gl) {
-      const uint4 w_lo = nw_lo, w_hi = nw_hi;
-      const float sf_lo = __half2float(__ushort_as_half(ns_lo)), sf_hi = __half2float(__ushort_as_half(ns_hi));
-      const uint32_t zc_lo = neg_zc(nz_lo), zc_hi = neg_zc(nz_hi);
-      if (gl + 1 < ng) {
-        const int gg = g0 + gl + 1;
-        nw_lo = ld_codes16(c_lo + (size_t)gg * 64);
-        nw_hi = ld_codes16(c_hi + (size_t)gg * 64);
-        ns_lo = ld_u16(s_lo + gg);
-        ns_hi = ld_u16(s_hi + gg);
-        nz_lo = ld_u16(z_lo + gg);
-        nz_hi = ld_u16(z_hi + gg);
-      }
-      float part[TB][4];
+    if (active) {
+      const uint32_t ts = (uint32_t)m.kc * 256u + 16u;
+      const uint8_t* xrow = smem + (size_t)buf * P.buf_bytes + (size_t)g * ts;
+#pragma unroll 1
+      for (int gl = 0; gl < it.ng; ++gl) {
+        if (fv) fetch(fslot);
+        cp_async_commit();
+        fslot = fslot + 1 == kSkRing ? 0 : fslot + 1;
+        cp_async_wait<kSkRing - 1>();  // this step's codes have landed
+        uint4 w_lo, w_hi;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(w_lo.x), "=r"(w_lo.y), "=r"(w_lo.z), "=r"(w_lo.w) : "r"(ring_me + cslot * kSlot) : "memory");
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(w_hi.x), "=r"(w_hi.y), "=r"(w_hi.z), "=r"(w_hi.w) : "r"(ring_me + cslot * kSlot + kSlot / 2) : "memory");
+        cslot = cslot + 1 == kSkRing ? 0 : cslot + 1;
+        const float sf_lo = __half2float(__ushort_as_half(ns_lo)), sf_hi = __half2float(__ushort_as_half(ns_hi));
+        const uint32_t zc_lo = neg_zc(nz_lo), zc_hi = neg_zc(nz_hi);
+        if (sv) load_meta();
+        float part[TB][4];
+        const uint32_t wl[4] = {w_lo.x, w_lo.y, w_lo.z, w_lo.w};
+        const uint32_t wh[4] = {w_hi.x, w_hi.y, w_hi.z, w_hi.w};
+        const uint8_t* xg = xrow + (size_t)gl * 256;
 #pragma unroll
-      for (int b = 0; b < TB; ++b) part[b][0] = part[b][1] = part[b][2] = part[b][3] = 0.f;
-      const uint32_t wl[4] = {w_lo.x, w_lo.y, w_lo.z, w_lo.w};
-      const uint32_t wh[4] = {w_hi.x, w_hi.y, w_hi.z, w_hi.w};
+        for (int w = 0; w < 4; ++w) {
+          const uint32_t a0 = pair_minus_z(wl[w], 0x0000u, zc_lo), a1 = pair_minus_z(wh[w], 0x0000u, zc_hi);
+          const uint32_t a2 = pair_minus_z(wl[w], 0x1111u, zc_lo), a3 = pair_minus_z(wh[w], 0x1111u, zc_hi);
+          const uint32_t e0 = pair_minus_z(wl[w], 0x2222u, zc_lo), e1 = pair_minus_z(wh[w], 0x2222u, zc_hi);
+          const uint32_t e2 = pair_minus_z(wl[w], 0x3333u, zc_lo), e3 = pair_minus_z(wh[w], 0x3333u, zc_hi);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint32_t a0 = pair_minus_z(wl[w], 0x0000u, zc_lo), a1 = pair_minus_z(wh[w], 0x0000u, zc_hi);
-        const uint32_t a2 = pair_minus_z(wl[w], 0x1111u, zc_lo), a3 = pair_minus_z(wh[w], 0x1111u, zc_hi);
-        const uint32_t e0 = pair_minus_z(wl[w], 0x2222u, zc_lo), e1 = pair_minus_z(wh[w], 0x2222u, zc_hi);
-        const uint32_t e2 = pair_minus_z(wl[w], 0x3333u, zc_lo), e3 = pair_minus_z(wh[w], 0x3333u, zc_hi);
-        const uint8_t* xo = xrow + (size_t)gl * 256 + xchunk_off((uint32_t)(4 * t + w));
+          for (int b = 0; b < TB; ++b) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(xg + xoff[w] + (size_t)(8 * b) * ts);
+            if (w == 0) mma16816_z(part[b], a0, a1, a2, a3, xv.x, xv.y);
+            else mma16816(part[b], a0, a1, a2, a3, xv.x, xv.y);
+            mma16816(part[b], e0, e1, e2, e3, xv.z, xv.w);
+          }
+        }
 #pragma unroll
         for (int b = 0; b < TB; ++b) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(xo + (size_t)(8 * b) * ts);
-          mma16816(part[b], a0, a1, a2, a3, xv.x, xv.y);
-          mma16816(part[b], e0, e1, e2, e3, xv.z, xv.w);
+          acc[b][0] = fmaf(sf_lo, part[b][0], acc[b][0]);
+          acc[b][1] = fmaf(sf_lo, part[b][1], acc[b][1]);
+          acc[b][2] = fmaf(sf_hi, part[b][2], acc[b][2]);
+          acc[b][3] = fmaf(sf_hi, part[b][3], acc[b][3]);
         }
       }
+      if (it.ch + 1 == m.nch) {
+        // C fragment: (row g, tokens 2t, 2t + 1) and (row g + 8, the same tokens)
+        const int ra = (it.ws + warp - m.slab_begin) * 16 + g, rb = ra + 8;
 #pragma unroll
-      for (int b = 0; b < TB; ++b) {
-        acc[b][0] = fmaf(sf_lo, part[b][0], acc[b][0]);
-        acc[b][1] = fmaf(sf_lo, part[b][1], acc[b][1]);
-        acc[b][2] = fmaf(sf_hi, part[b][2], acc[b][2]);
-        acc[b][3] = fmaf(sf_hi, part[b][3], acc[b][3]);
-      }
-    }
-
-    if (cur.ch + 1 == Mt.nch) {
-      // C fragment: (row g, tokens 2t, 2t + 1) and (row g + 8, the same tokens)
-      const int ra = n0 + g, rb = n0 + g + 8;
-#pragma unroll
-      for (int b = 0; b < TB; ++b) {
-        const int m = 8 * b + 2 * t;
-        if (m < M) {
-          if (ra < Mt.N) Mt.y[(size_t)m * Mt.N + ra] = __half_as_ushort(__float2half_rn(acc[b][0]));
-          if (rb < Mt.N) Mt.y[(size_t)m * Mt.N + rb] = __half_as_ushort(__float2half_rn(acc[b][2]));
+        for (int b = 0; b < TB; ++b) {
+          const int mt = 8 * b + 2 * t;
+          if (mt < M) {
+            if (ra < m.N) m.y[(size_t)mt * m.N + ra] = __half_as_ushort(__float2half_rn(acc[b][0]));
+            if (rb < m.N) m.y[(size_t)mt * m.N + rb] = __half_as_ushort(__float2half_rn(acc[b][2]));
+          }
+          if (mt + 1 < M) {
+            if (ra < m.N) m.y[(size_t)(mt + 1) * m.N + ra] = __half_as_ushort(__float2half_rn(acc[b][1]));
+            if (rb < m.N) m.y[(size_t)(mt + 1) * m.N + rb] = __half_as_ushort(__float2half_rn(acc[b][3]));
+          }
+          acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
         }
-        if (m + 1 < M) {
-          if (ra < Mt.N) Mt.y[(size_t)(m + 1) * Mt.N + ra] = __half_as_ushort(__float2half_rn(acc[b][1]));
-          if (rb < Mt.N) Mt.y[(size_t)(m + 1) * Mt.N + rb] = __half_as_ushort(__float2half_rn(acc[b][3]));
-        }
-        acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
       }
+    } else if (restage) {
+      cp_async_commit();  // the staging copies alone
     }
-    cur = nxt;
+    if (!has_next) break;
+    if (restage) {
+      // This thread's staging copies rode in the group committed at the item's first step,
+      // which the per-step waits have covered once the item had kSkRing steps; otherwise
+      // wait for it here. Then every thread's copies are visible after the barrier, and no
+      // warp reads the buffer the next restage will overwrite.
+      if (!active) cp_async_wait<0>();
+      else if (it.ng < kSkRing) cp_async_wait_upto(it.ng - 1);
+      __syncthreads();
+      buf ^= 1;
+    }
+    it = nx;
   }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  cp_async_wait<0>();
 }
 
 // ---- host side -----------------------------------------------------------------------
@@ -249,31 +389,18 @@ static int tb_for(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : 4; }
 
 int skinny_plan(SkParams& p, int count, const SkDesc* d, int M) {
   if (count < 1 || count > kSkMaxMats || M < 1 || M > kSkMaxM) return 0;
-  const int tb = tb_for(M);
-  // one buffer: 8 TB token rows of kc * 256 + 16 bytes; two buffers per CTA
-  const int kc_max = ((kSkSmemPerCta / 2) / (8 * tb) - 16) / 256;
+  const int nt = 8 * tb_for(M);
+  // two activation buffers of nt token rows, kc * 256 + 16 bytes each, beside the codes ring
+  const int kc_max = (((kSkSmemMax - kSkRingBytes) / 2) / nt - 16) / 256;
   if (kc_max < 1) return 0;
-  static thread_local int order[kSkMaxMats];
-  for (int i = 0; i < count; ++i) {
-    if (((uintptr_t)d[i].codes & 15) || ((uintptr_t)d[i].x & 15) || ((uintptr_t)d[i].scale & 1) ||
-        ((uintptr_t)d[i].zero & 1) || !d[i].zero)
-      return 0;
-    order[i] = i;
-  }
-  for (int i = 1; i < count; ++i) {  // stable insertion sort by K, descending
-    const int v = order[i];
-    int j = i;
-    while (j > 0 && d[order[j - 1]].K < d[v].K) {
-      order[j] = order[j - 1];
-      --j;
-    }
-    order[j] = v;
-  }
-  int64_t units = 0;
+  int64_t slabs = 0, cost = 0;
   int kc_used = 1;
-  for (int j = 0; j < count; ++j) {
-    const SkDesc& s = d[order[j]];
-    SkMat& m = p.m[j];
+  for (int i = 0; i < count; ++i) {
+    const SkDesc& s = d[i];
+    if (((uintptr_t)s.codes & 15) || ((uintptr_t)s.x & 15) || ((uintptr_t)s.scale & 1) || !s.zero ||
+        ((uintptr_t)s.zero & 1))
+      return 0;
+    SkMat& m = p.m[i];
     m.codes = static_cast<const uint8_t*>(s.codes);
     m.scale = s.scale;
     m.zero = s.zero;
@@ -281,19 +408,24 @@ int skinny_plan(SkParams& p, int count, const SkDesc* d, int M) {
     m.y = s.y;
     m.N = (int)s.N;
     m.K = (int)s.K;
-    const int G = (int)(s.K / kGroup);
-    m.nch = (G + kc_max - 1) / kc_max;
-    m.kc = (G + m.nch - 1) / m.nch;
+    m.G = (int)(s.K / kGroup);
+    m.nch = (m.G + kc_max - 1) / kc_max;
+    m.kc = (m.G + m.nch - 1) / m.nch;
     kc_used = m.kc > kc_used ? m.kc : kc_used;
-    m.unit_begin = (int)units;
-    units += (s.N + kSkUnitRows - 1) / kSkUnitRows;
-    if (units > INT_MAX) return 0;
+    const int64_t ns = (s.N + 15) / 16;
+    m.slab_begin = (int)slabs;
+    m.cost_begin = cost;
+    slabs += ns;
+    cost += ns * m.G;
+    if (slabs > INT_MAX) return 0;
+    m.slab_end = (int)slabs;
   }
   p.count = count;
   p.M = M;
-  p.total_units = (int)units;
-  p.buf_bytes = 8 * tb * (kc_used * 256 + 16);
-  return 2 * p.buf_bytes;
+  p.total_slabs = (int)slabs;
+  p.total_cost = cost;
+  p.buf_bytes = nt * (kc_used * 256 + 16);
+  return 2 * p.buf_bytes + kSkRingBytes;
 }
 
 template <int TB>
@@ -305,20 +437,20 @@ static cudaError_t launch_tb(const SkParams& p, int smem, cudaStream_t stream) {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_done[dev]) {
     e = cudaFuncSetAttribute(gemm_skinny_kernel<TB, kSkMaxMats>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSkSmemPerCta);
+                             kSkSmemMax);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const int grid = p.total_units < kSkCtasPerSm * sms ? p.total_units : kSkCtasPerSm * sms;
-  gemm_skinny_kernel<TB, kSkMaxMats><<<grid, kThreads, smem, stream>>>(p);
+  const int grid = p.total_slabs < sms ? p.total_slabs : sms;  // one CTA per SM
+  gemm_skinny_kernel<TB, kSkMaxMats><<<grid, kSkThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_skinny(const SkParams& p, int smem, cudaStream_t stream) {
-  if (smem <= 0 || smem > kSkSmemPerCta || p.total_units < 1) return cudaErrorInvalidValue;
+  if (smem <= 0 || smem > kSkSmemMax || p.total_slabs < 1) return cudaErrorInvalidValue;
   switch (tb_for(p.M)) {
     case 1: return launch_tb<1>(p, smem, stream);
     case 2: return launch_tb<2>(p, smem, stream);

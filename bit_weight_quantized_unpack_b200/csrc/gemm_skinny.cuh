@@ -7,8 +7,8 @@
 
 namespace wq {
 
-constexpr int kSkWarps = 8;           // warps per CTA, one 16-row weight slab each
-constexpr int kSkUnitRows = 16 * kSkWarps;  // weight rows per unit of work (128)
+constexpr int kSkWarps = 16;          // warps per CTA (one CTA per SM), one 16-row slab each
+constexpr int kSkThreads = 32 * kSkWarps;
 #ifndef WQ_SK_MIN_M
 #define WQ_SK_MIN_M 5
 #endif
@@ -16,19 +16,23 @@ constexpr int kSkMinM = WQ_SK_MIN_M;  // wq_gemm / wq_linear_set use this kernel
                                       // this M (below it the streaming kernel is faster) ...
 constexpr int kSkMaxM = 32;           // ... up to this M (tokens per product)
 constexpr int kSkMaxMats = 256;
-constexpr int kSkCtasPerSm = 2;       // register budget of the launch bounds
-constexpr int kSkSmemPerCta = 112 * 1024;  // two activation buffers
+constexpr int kSkRing = 4;            // code groups in flight per thread (cp.async ring)
+constexpr int kSkRingBytes = kSkRing * 2 * kSkThreads * 16;  // 64 KB
+constexpr int kSkSmemMax = 232448;    // dynamic shared memory of one CTA (227 KB)
 
-// One matrix; its units are [unit_begin, unit_begin + ceil(N / 128)). The activations of a
-// unit are staged in chunks of kc groups (nch chunks, the last one possibly shorter).
+// One matrix: slabs [slab_begin, slab_end) of the launch (16 weight rows each, the last one
+// possibly short), at cost positions cost_begin + j * G (cost = 128-weight groups). The
+// activations of a window of slabs are staged in chunks of kc groups (nch chunks, the last
+// one possibly shorter).
 struct SkMat {
   const uint8_t* codes;    // int4 codes, bytes [N, K/2]
   const uint16_t* scale;   // fp16 [N, K/128]
   const uint16_t* zero;    // fp16 [N, K/128]
   const uint16_t* x;       // fp16 [M, K], 16-byte aligned
   uint16_t* y;             // fp16 [M, N]
-  int N, K;
-  int unit_begin;
+  int64_t cost_begin;
+  int N, K, G;
+  int slab_begin, slab_end;
   int nch, kc;
 };
 
@@ -36,8 +40,9 @@ template <int CAP>
 struct SkParamsT {
   int count;
   int M;
-  int total_units;
+  int total_slabs;
   int buf_bytes;           // bytes of one activation buffer
+  int64_t total_cost;
   SkMat m[CAP];
 };
 using SkParams = SkParamsT<kSkMaxMats>;
@@ -51,9 +56,9 @@ struct SkDesc {
   int64_t N, K;
 };
 
-// Fills p for `count` int4 matrices multiplied by M tokens (1 <= M <= kSkMaxM), ordered by
-// K, largest first, and returns the dynamic shared memory of a CTA, or 0 if the kernel
-// cannot serve the set (alignment, or more than kSkMaxMats matrices).
+// Fills p for `count` int4 matrices multiplied by M tokens (1 <= M <= kSkMaxM) and returns
+// the dynamic shared memory of a CTA, or 0 if the kernel cannot serve the set (alignment, or
+// more than kSkMaxMats matrices).
 int skinny_plan(SkParams& p, int count, const SkDesc* d, int M);
 cudaError_t launch_gemm_skinny(const SkParams& p, int smem, cudaStream_t stream);
 
