@@ -82,12 +82,23 @@ __device__ __forceinline__ uint32_t neg_zc(uint16_t zb) {
 // stride of 16 (mod 128) bytes.
 __device__ __forceinline__ uint32_t xchunk_off(uint32_t c) { return (c ^ (((c >> 3) & 1u) << 1)) << 4; }
 
+// Per-step ring traffic: these statements are volatile, so they keep their order among
+// themselves (copy, commit, wait, read back); they carry no memory clobber, so that the
+// compiler may schedule the step's other work across them. (The activation buffer a step
+// reads is never the one being written; restaging is ordered by barriers.)
 __device__ __forceinline__ void cp_async16_l2(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(dst), "l"(src));
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+__device__ __forceinline__ void cp_async_commit_step() { asm volatile("cp.async.commit_group;"); }
+
+template <int RING>
+__device__ __forceinline__ void cp_async_wait_step() { asm volatile("cp.async.wait_group %0;" ::"n"(RING - 1)); }
+
+__device__ __forceinline__ uint4 lds_ring(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -95,13 +106,14 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// wait until at most n (0 <= n < kSkRing) of this thread's newest copy groups are pending
+// wait until at most n (0 <= n < 6) of this thread's newest copy groups are pending
 __device__ __forceinline__ void cp_async_wait_upto(int n) {
-  static_assert(kSkRing == 4, "one case per ring depth");
   if (n <= 0) cp_async_wait<0>();
   else if (n == 1) cp_async_wait<1>();
   else if (n == 2) cp_async_wait<2>();
-  else cp_async_wait<3>();
+  else if (n == 3) cp_async_wait<3>();
+  else if (n == 4) cp_async_wait<4>();
+  else cp_async_wait<5>();
 }
 
 // d = A * B with a zero accumulator (first MMA of a group)
@@ -112,8 +124,8 @@ __device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-// A position in a CTA's work: item = window [ws, we) of slabs (one per warp) of matrix mi and
-// activation chunk ch (groups g0 .. g0 + ng - 1); step gl = group g0 + gl of the item.
+// A position in a CTA's work: item = window [ws, we) of slabs of matrix mi (warp w takes
+// slabs ws + w, ws + w + 16, ...) and activation chunk ch (groups g0 .. g0 + ng - 1).
 struct Walk {
   int ws, we, mi, ch, g0, ng, gl;
 };
@@ -121,7 +133,7 @@ struct Walk {
 template <int CAP>
 __device__ __forceinline__ void item_fill(const SkParamsT<CAP>& P, Walk& w, int hi) {
   const SkMat& m = P.m[w.mi];
-  w.we = min(min(w.ws + kSkWarps, m.slab_end), hi);
+  w.we = min(min(w.ws + m.span, m.slab_end), hi);
   w.g0 = w.ch * m.kc;
   w.ng = min(m.kc, m.G - w.g0);
 }
@@ -168,6 +180,7 @@ __device__ __forceinline__ int mat_of_slab(const SkParamsT<CAP>& P, int s) {
 
 template <int TB, int CAP>
 __global__ void __launch_bounds__(kSkThreads, 1) gemm_skinny_kernel(const __grid_constant__ SkParamsT<CAP> P) {
+  constexpr int kRing = sk_ring(TB);
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -205,85 +218,84 @@ __global__ void __launch_bounds__(kSkThreads, 1) gemm_skinny_kernel(const __grid
   cp_async_wait<0>();
   __syncthreads();
 
-  // Fetch cursor (kSkRing - 1 steps ahead of the compute) and metadata cursor (one step
-  // ahead). Each keeps the sources of its next step in registers and walks them with pointer
-  // bumps; the item bookkeeping runs only when it moves to another item.
+  // Fetch cursor (kRing - 1 steps ahead of the compute) and metadata cursor (one step
+  // ahead) over this warp's steps: items in order, in each the warp's slabs in order, in each
+  // slab the chunk's groups. Each keeps the source of its next step in registers and the
+  // steps left in its slab; the slab and item bookkeeping runs only when that count runs out.
   Walk f = it;
   bool fv = true;
   while (warp >= f.we - f.ws)
     if (!item_next(P, f, hi)) { fv = false; break; }
   Walk sc = f;
   bool sv = fv;
+  int fs = f.ws + warp, ss = fs;  // the cursors' current slabs
   const uint8_t* fp_lo = nullptr;
   const uint8_t* fp_hi = nullptr;
-  const uint16_t* fm = nullptr;
-  auto fetch_item = [&]() {
+  int f_left = 0;  // steps left in the fetch cursor's slab (0: no more steps)
+  auto fetch_slab = [&]() {
     const SkMat& m = P.m[f.mi];
-    const int r0 = (f.ws + warp - m.slab_begin) * 16 + g;
-    const int rl = min(r0, m.N - 1), rh = min(r0 + 8, m.N - 1);
-    fp_lo = m.codes + (size_t)rl * (m.K / 2) + (size_t)f.g0 * 64 + 16 * t;
-    fp_hi = m.codes + (size_t)rh * (m.K / 2) + (size_t)f.g0 * 64 + 16 * t;
-    // the metadata value this lane prefetches: t = 0, 1: scale of row g, g + 8; 2, 3: zero
-    fm = ((t & 2) ? m.zero : m.scale) + (size_t)((t & 1) ? rh : rl) * m.G + f.g0;
+    const int r0 = (fs - m.slab_begin) * 16 + g;
+    fp_lo = m.codes + (size_t)min(r0, m.N - 1) * (m.K / 2) + (size_t)f.g0 * 64 + 16 * t;
+    fp_hi = m.codes + (size_t)min(r0 + 8, m.N - 1) * (m.K / 2) + (size_t)f.g0 * 64 + 16 * t;
+    f_left = f.ng;
   };
-  if (fv) fetch_item();
-  auto fetch = [&](uint32_t slot) {
-    cp_async16_l2(ring_me + slot * kSlot, fp_lo);
-    cp_async16_l2(ring_me + slot * kSlot + kSlot / 2, fp_hi);
-    prefetch_l2(fm);
-    if (++f.gl < f.ng) {
+  if (fv) fetch_slab();
+  const uint32_t ring_first = ring_me, ring_last = ring_me + (uint32_t)(kRing - 1) * kSlot;
+  uint32_t fslot = ring_first, cslot = ring_first;
+  auto fetch = [&]() {
+    if (f_left > 0) {
+      cp_async16_l2(fslot, fp_lo);
+      cp_async16_l2(fslot + kSlot / 2, fp_hi);
       fp_lo += 64;
       fp_hi += 64;
-      fm += 1;
-    } else {
-      f.gl = 0;
-      do {
-        if (!item_next(P, f, hi)) { fv = false; break; }
-      } while (warp >= f.we - f.ws);
-      if (fv) fetch_item();
+      if (--f_left == 0) {
+        fs += kSkWarps;
+        if (fs >= f.we) {
+          f.gl = 0;
+          do {
+            if (!item_next(P, f, hi)) { fv = false; break; }
+          } while (warp >= f.we - f.ws);
+          fs = f.ws + warp;
+        }
+        if (fv) fetch_slab();
+      }
     }
+    cp_async_commit_step();
+    fslot = fslot == ring_last ? ring_first : fslot + kSlot;
   };
-  uint32_t fslot = 0;
 #pragma unroll 1
-  for (int d = 0; d < kSkRing - 1; ++d) {
-    if (fv) fetch(fslot);
-    cp_async_commit();
-    fslot = fslot + 1 == kSkRing ? 0 : fslot + 1;
-  }
+  for (int d = 0; d < kRing - 1; ++d) fetch();
 
-  // metadata of the next step, in registers
-  const uint16_t* ms_lo = nullptr;
-  const uint16_t* ms_hi = nullptr;
-  const uint16_t* mz_lo = nullptr;
-  const uint16_t* mz_hi = nullptr;
-  auto meta_item = [&]() {
+  // Metadata: lane (g, t) loads one value per step (t = 0, 1: scale of row g, g + 8;
+  // t = 2, 3: zero of row g, g + 8), one step ahead; shuffles within the lane group hand
+  // each lane all four.
+  const uint16_t* mp = nullptr;
+  int m_left = 0;
+  auto meta_slab = [&]() {
     const SkMat& m = P.m[sc.mi];
-    const int r0 = (sc.ws + warp - m.slab_begin) * 16 + g;
-    const size_t il = (size_t)min(r0, m.N - 1) * m.G + sc.g0;
-    const size_t ih = (size_t)min(r0 + 8, m.N - 1) * m.G + sc.g0;
-    ms_lo = m.scale + il;
-    ms_hi = m.scale + ih;
-    mz_lo = m.zero + il;
-    mz_hi = m.zero + ih;
+    const int r = min((ss - m.slab_begin) * 16 + g + ((t & 1) ? 8 : 0), m.N - 1);
+    mp = ((t & 2) ? m.zero : m.scale) + (size_t)r * m.G + sc.g0;
+    m_left = sc.ng;
   };
-  uint16_t ns_lo = 0, ns_hi = 0, nz_lo = 0, nz_hi = 0;
+  uint32_t nmeta = 0;
   auto load_meta = [&]() {
-    ns_lo = ld_u16(ms_lo + sc.gl);
-    ns_hi = ld_u16(ms_hi + sc.gl);
-    nz_lo = ld_u16(mz_lo + sc.gl);
-    nz_hi = ld_u16(mz_hi + sc.gl);
-    if (++sc.gl == sc.ng) {
-      sc.gl = 0;
-      do {
-        if (!item_next(P, sc, hi)) { sv = false; break; }
-      } while (warp >= sc.we - sc.ws);
-      if (sv) meta_item();
+    if (m_left > 0) {
+      nmeta = ld_u16(mp);
+      ++mp;
+      if (--m_left == 0) {
+        ss += kSkWarps;
+        if (ss >= sc.we) {
+          do {
+            if (!item_next(P, sc, hi)) { sv = false; break; }
+          } while (warp >= sc.we - sc.ws);
+          ss = sc.ws + warp;
+        }
+        if (sv) meta_slab();
+      }
     }
   };
-  if (sv) {
-    meta_item();
-    load_meta();
-  }
+  if (sv) meta_slab();
+  load_meta();
 
   uint32_t xoff[4];
 #pragma unroll
@@ -292,76 +304,78 @@ __global__ void __launch_bounds__(kSkThreads, 1) gemm_skinny_kernel(const __grid
   float acc[TB][4];
 #pragma unroll
   for (int b = 0; b < TB; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
-  uint32_t cslot = 0;
   int buf = 0;
 
   for (;;) {
     const SkMat& m = P.m[it.mi];
-    const bool active = warp < it.we - it.ws;
+    const int nmine = warp < it.we - it.ws ? (it.we - it.ws - warp + kSkWarps - 1) / kSkWarps : 0;
     Walk nx = it;
     const bool has_next = item_next(P, nx, hi);
     const bool restage = has_next && (nx.mi != it.mi || nx.ch != it.ch);
     if (restage) stage_x(nx, buf ^ 1);  // these copies join this thread's next commit
 
-    if (active) {
+    if (nmine > 0) {
       const uint32_t ts = (uint32_t)m.kc * 256u + 16u;
       const uint8_t* xrow = smem + (size_t)buf * P.buf_bytes + (size_t)g * ts;
 #pragma unroll 1
-      for (int gl = 0; gl < it.ng; ++gl) {
-        if (fv) fetch(fslot);
-        cp_async_commit();
-        fslot = fslot + 1 == kSkRing ? 0 : fslot + 1;
-        cp_async_wait<kSkRing - 1>();  // this step's codes have landed
-        uint4 w_lo, w_hi;
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(w_lo.x), "=r"(w_lo.y), "=r"(w_lo.z), "=r"(w_lo.w) : "r"(ring_me + cslot * kSlot) : "memory");
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(w_hi.x), "=r"(w_hi.y), "=r"(w_hi.z), "=r"(w_hi.w) : "r"(ring_me + cslot * kSlot + kSlot / 2) : "memory");
-        cslot = cslot + 1 == kSkRing ? 0 : cslot + 1;
-        const float sf_lo = __half2float(__ushort_as_half(ns_lo)), sf_hi = __half2float(__ushort_as_half(ns_hi));
-        const uint32_t zc_lo = neg_zc(nz_lo), zc_hi = neg_zc(nz_hi);
-        if (sv) load_meta();
-        float part[TB][4];
-        const uint32_t wl[4] = {w_lo.x, w_lo.y, w_lo.z, w_lo.w};
-        const uint32_t wh[4] = {w_hi.x, w_hi.y, w_hi.z, w_hi.w};
-        const uint8_t* xg = xrow + (size_t)gl * 256;
+      for (int k = 0; k < nmine; ++k) {
+#pragma unroll 1
+        for (int gl = 0; gl < it.ng; ++gl) {
+          fetch();
+          cp_async_wait_step<kRing>();  // this step's codes have landed
+          const uint4 w_lo = lds_ring(cslot), w_hi = lds_ring(cslot + kSlot / 2);
+          cslot = cslot == ring_last ? ring_first : cslot + kSlot;
+          const uint32_t meta = nmeta;
+          load_meta();
+          const int q = lane & ~3;
+          const uint16_t s_lo = (uint16_t)__shfl_sync(0xFFFFFFFFu, meta, q);
+          const uint16_t s_hi = (uint16_t)__shfl_sync(0xFFFFFFFFu, meta, q + 1);
+          const uint16_t z_lo = (uint16_t)__shfl_sync(0xFFFFFFFFu, meta, q + 2);
+          const uint16_t z_hi = (uint16_t)__shfl_sync(0xFFFFFFFFu, meta, q + 3);
+          const float sf_lo = __half2float(__ushort_as_half(s_lo)), sf_hi = __half2float(__ushort_as_half(s_hi));
+          const uint32_t zc_lo = neg_zc(z_lo), zc_hi = neg_zc(z_hi);
+          float part[TB][4];
+          const uint32_t wl[4] = {w_lo.x, w_lo.y, w_lo.z, w_lo.w};
+          const uint32_t wh[4] = {w_hi.x, w_hi.y, w_hi.z, w_hi.w};
+          const uint8_t* xg = xrow + (size_t)gl * 256;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const uint32_t a0 = pair_minus_z(wl[w], 0x0000u, zc_lo), a1 = pair_minus_z(wh[w], 0x0000u, zc_hi);
-          const uint32_t a2 = pair_minus_z(wl[w], 0x1111u, zc_lo), a3 = pair_minus_z(wh[w], 0x1111u, zc_hi);
-          const uint32_t e0 = pair_minus_z(wl[w], 0x2222u, zc_lo), e1 = pair_minus_z(wh[w], 0x2222u, zc_hi);
-          const uint32_t e2 = pair_minus_z(wl[w], 0x3333u, zc_lo), e3 = pair_minus_z(wh[w], 0x3333u, zc_hi);
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t a0 = pair_minus_z(wl[w], 0x0000u, zc_lo), a1 = pair_minus_z(wh[w], 0x0000u, zc_hi);
+            const uint32_t a2 = pair_minus_z(wl[w], 0x1111u, zc_lo), a3 = pair_minus_z(wh[w], 0x1111u, zc_hi);
+            const uint32_t e0 = pair_minus_z(wl[w], 0x2222u, zc_lo), e1 = pair_minus_z(wh[w], 0x2222u, zc_hi);
+            const uint32_t e2 = pair_minus_z(wl[w], 0x3333u, zc_lo), e3 = pair_minus_z(wh[w], 0x3333u, zc_hi);
+#pragma unroll
+            for (int b = 0; b < TB; ++b) {
+              const uint4 xv = *reinterpret_cast<const uint4*>(xg + xoff[w] + (size_t)(8 * b) * ts);
+              if (w == 0) mma16816_z(part[b], a0, a1, a2, a3, xv.x, xv.y);
+              else mma16816(part[b], a0, a1, a2, a3, xv.x, xv.y);
+              mma16816(part[b], e0, e1, e2, e3, xv.z, xv.w);
+            }
+          }
 #pragma unroll
           for (int b = 0; b < TB; ++b) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(xg + xoff[w] + (size_t)(8 * b) * ts);
-            if (w == 0) mma16816_z(part[b], a0, a1, a2, a3, xv.x, xv.y);
-            else mma16816(part[b], a0, a1, a2, a3, xv.x, xv.y);
-            mma16816(part[b], e0, e1, e2, e3, xv.z, xv.w);
+            acc[b][0] = fmaf(sf_lo, part[b][0], acc[b][0]);
+            acc[b][1] = fmaf(sf_lo, part[b][1], acc[b][1]);
+            acc[b][2] = fmaf(sf_hi, part[b][2], acc[b][2]);
+            acc[b][3] = fmaf(sf_hi, part[b][3], acc[b][3]);
           }
         }
+        if (it.ch + 1 == m.nch) {
+          // C fragment: (row g, tokens 2t, 2t + 1) and (row g + 8, the same tokens)
+          const int ra = (it.ws + warp + kSkWarps * k - m.slab_begin) * 16 + g, rb = ra + 8;
 #pragma unroll
-        for (int b = 0; b < TB; ++b) {
-          acc[b][0] = fmaf(sf_lo, part[b][0], acc[b][0]);
-          acc[b][1] = fmaf(sf_lo, part[b][1], acc[b][1]);
-          acc[b][2] = fmaf(sf_hi, part[b][2], acc[b][2]);
-          acc[b][3] = fmaf(sf_hi, part[b][3], acc[b][3]);
-        }
-      }
-      if (it.ch + 1 == m.nch) {
-        // C fragment: (row g, tokens 2t, 2t + 1) and (row g + 8, the same tokens)
-        const int ra = (it.ws + warp - m.slab_begin) * 16 + g, rb = ra + 8;
-#pragma unroll
-        for (int b = 0; b < TB; ++b) {
-          const int mt = 8 * b + 2 * t;
-          if (mt < M) {
-            if (ra < m.N) m.y[(size_t)mt * m.N + ra] = __half_as_ushort(__float2half_rn(acc[b][0]));
-            if (rb < m.N) m.y[(size_t)mt * m.N + rb] = __half_as_ushort(__float2half_rn(acc[b][2]));
+          for (int b = 0; b < TB; ++b) {
+            const int mt = 8 * b + 2 * t;
+            if (mt < M) {
+              if (ra < m.N) m.y[(size_t)mt * m.N + ra] = __half_as_ushort(__float2half_rn(acc[b][0]));
+              if (rb < m.N) m.y[(size_t)mt * m.N + rb] = __half_as_ushort(__float2half_rn(acc[b][2]));
+            }
+            if (mt + 1 < M) {
+              if (ra < m.N) m.y[(size_t)(mt + 1) * m.N + ra] = __half_as_ushort(__float2half_rn(acc[b][1]));
+              if (rb < m.N) m.y[(size_t)(mt + 1) * m.N + rb] = __half_as_ushort(__float2half_rn(acc[b][3]));
+            }
+            acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
           }
-          if (mt + 1 < M) {
-            if (ra < m.N) m.y[(size_t)(mt + 1) * m.N + ra] = __half_as_ushort(__float2half_rn(acc[b][1]));
-            if (rb < m.N) m.y[(size_t)(mt + 1) * m.N + rb] = __half_as_ushort(__float2half_rn(acc[b][3]));
-          }
-          acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
         }
       }
     } else if (restage) {
@@ -369,12 +383,13 @@ __global__ void __launch_bounds__(kSkThreads, 1) gemm_skinny_kernel(const __grid
     }
     if (!has_next) break;
     if (restage) {
-      // This thread's staging copies rode in the group committed at the item's first step,
-      // which the per-step waits have covered once the item had kSkRing steps; otherwise
-      // wait for it here. Then every thread's copies are visible after the barrier, and no
-      // warp reads the buffer the next restage will overwrite.
-      if (!active) cp_async_wait<0>();
-      else if (it.ng < kSkRing) cp_async_wait_upto(it.ng - 1);
+      // This thread's staging copies rode in the group committed at its first step of the
+      // item, which the per-step waits have covered once the item had as many of its steps as the ring has slots;
+      // otherwise wait for it here. Then every thread's copies are visible after the
+      // barrier, and no warp still reads the buffer the next restage will overwrite.
+      const int steps = nmine * it.ng;
+      if (steps == 0) cp_async_wait<0>();
+      else if (steps < kRing) cp_async_wait_upto(steps - 1);
       __syncthreads();
       buf ^= 1;
     }
@@ -391,7 +406,7 @@ int skinny_plan(SkParams& p, int count, const SkDesc* d, int M) {
   if (count < 1 || count > kSkMaxMats || M < 1 || M > kSkMaxM) return 0;
   const int nt = 8 * tb_for(M);
   // two activation buffers of nt token rows, kc * 256 + 16 bytes each, beside the codes ring
-  const int kc_max = (((kSkSmemMax - kSkRingBytes) / 2) / nt - 16) / 256;
+  const int kc_max = (((kSkSmemMax - sk_ring_bytes(tb_for(M))) / 2) / nt - 16) / 256;
   if (kc_max < 1) return 0;
   int64_t slabs = 0, cost = 0;
   int kc_used = 1;
@@ -411,6 +426,7 @@ int skinny_plan(SkParams& p, int count, const SkDesc* d, int M) {
     m.G = (int)(s.K / kGroup);
     m.nch = (m.G + kc_max - 1) / kc_max;
     m.kc = (m.G + m.nch - 1) / m.nch;
+    m.span = kSkWarps * (m.nch == 1 ? kSkSpanOne : 1);
     kc_used = m.kc > kc_used ? m.kc : kc_used;
     const int64_t ns = (s.N + 15) / 16;
     m.slab_begin = (int)slabs;
@@ -425,7 +441,7 @@ int skinny_plan(SkParams& p, int count, const SkDesc* d, int M) {
   p.total_slabs = (int)slabs;
   p.total_cost = cost;
   p.buf_bytes = nt * (kc_used * 256 + 16);
-  return 2 * p.buf_bytes + kSkRingBytes;
+  return 2 * p.buf_bytes + sk_ring_bytes(tb_for(M));
 }
 
 template <int TB>

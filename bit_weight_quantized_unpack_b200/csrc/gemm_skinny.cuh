@@ -16,14 +16,20 @@ constexpr int kSkMinM = WQ_SK_MIN_M;  // wq_gemm / wq_linear_set use this kernel
                                       // this M (below it the streaming kernel is faster) ...
 constexpr int kSkMaxM = 32;           // ... up to this M (tokens per product)
 constexpr int kSkMaxMats = 256;
-constexpr int kSkRing = 4;            // code groups in flight per thread (cp.async ring)
-constexpr int kSkRingBytes = kSkRing * 2 * kSkThreads * 16;  // 64 KB
+// code groups in flight per thread (cp.async ring of 16 KB slots): six for up to 16 tokens;
+// four for more, whose activation chunks need the room
+__host__ __device__ constexpr int sk_ring(int tb) { return tb >= 4 ? 4 : 6; }
+__host__ __device__ constexpr int sk_ring_bytes(int tb) { return sk_ring(tb) * 2 * kSkThreads * 16; }
+constexpr int kSkSpanOne = 8;         // slabs per warp and window when the activations of a
+                                      // matrix fit one chunk
 constexpr int kSkSmemMax = 232448;    // dynamic shared memory of one CTA (227 KB)
 
 // One matrix: slabs [slab_begin, slab_end) of the launch (16 weight rows each, the last one
-// possibly short), at cost positions cost_begin + j * G (cost = 128-weight groups). The
-// activations of a window of slabs are staged in chunks of kc groups (nch chunks, the last
-// one possibly shorter).
+// possibly short), at cost positions cost_begin + j * G (cost = 128-weight groups). Its
+// slabs are taken in windows of up to `span` slabs (warp w: slabs w, w + 16, ...), and the
+// activations of a window are staged in chunks of kc groups (nch chunks, the last one
+// possibly shorter); with more than one chunk a window holds one slab per warp, whose sums
+// stay in registers across the chunks.
 struct SkMat {
   const uint8_t* codes;    // int4 codes, bytes [N, K/2]
   const uint16_t* scale;   // fp16 [N, K/128]
@@ -33,7 +39,7 @@ struct SkMat {
   int64_t cost_begin;
   int N, K, G;
   int slab_begin, slab_end;
-  int nch, kc;
+  int nch, kc, span;
 };
 
 template <int CAP>
