@@ -28,12 +28,18 @@
 // multiplies exact integer weights by the fp16 activations; the group scale is applied in
 // fp32 to each group's MMA sum. Only fp32 adds and the final fp16 store round.
 //
-// Work: units of 128 weight rows x all of K (eight warps, one 16-row slab each), ordered by
-// K (largest first) and dealt to CTAs round robin. The activations of a unit are staged in
-// shared memory (cp.async) in chunks of up to kc groups, two buffers, the next chunk's copy
-// in flight while the current one is used. Codes and metadata go straight from global
-// memory into registers one group ahead, with a 256-byte L2 fetch size so that a row's next
-// groups arrive with the current one.
+// Work: one CTA of 16 warps per SM. CTA b takes the contiguous range of slabs (16 rows x all
+// of K) whose cost (128-weight groups) falls in its 1/gridDim share of the set, walked in
+// windows: warp w takes slabs w, w + 16, ... of a window (up to 8 each when the matrix's
+// activations fit one chunk; one when they need several, whose sums stay in registers
+// across the chunks). The activations of a window are staged in shared memory with cp.async
+// in chunks of up to kc groups (two buffers), restaged only when the matrix or the chunk
+// changes. Codes travel through a per-thread cp.async ring in shared memory, several groups
+// deep, with a 256-byte L2 fetch size so that a row's next groups come with the current one;
+// the thread's copies form one commit group per compute step, and a restaged chunk's copies
+// ride in the group of the item's first step, so the per-step waits cover them too. Each
+// lane loads one of its lane group's four scale / zero values one step ahead; shuffles share
+// them.
 #include <climits>
 
 #include "common.cuh"
