@@ -262,7 +262,7 @@ def bench_7b_set(args, pk):
 
 def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 32, 64, 512, 2048)):
     """Batch sweep on the 0.5B set: M tokens through all 169 matrices in one wq_linear_set
-    call per pass (one streaming launch for M <= 4, one skinny-batch launch for 5 <= M <= 32,
+    call per pass (one skinny-batch launch for 2 <= M <= 32,
     tensor-core launches of up to 80 matrices for larger M). The set's 262 MB exceed L2."""
     from bit_weight_quantized_unpack_b200 import wq
     wl = workloads.WORKLOADS[4]
@@ -292,7 +292,7 @@ def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 32, 64, 512, 2048)):
         out[f"gemm_set_M{M}"] = {"ms": ms, "TFLOPS": flops / ms / 1e9,
                                  "frac_tensor": flops / ms / 1e9 / pk["bf16_tflops"],
                                  "weight_GBps": gbs, "frac_hbm": gbs / pk["hbm_gbs"],
-                                 "kernel": ("gemv_stream_kernel" if M <= 4 else
+                                 "kernel": ("gemv_stream_kernel" if M == 1 else
                                             "gemm_skinny_kernel" if M <= 32 else "gemm_tc_int4_kernel"),
                                  "launches_per_pass": (len(mats) + 79) // 80 if M > 32 else 1}
         del X, Y

@@ -10,10 +10,10 @@ namespace wq {
 constexpr int kSkWarps = 16;          // warps per CTA (one CTA per SM), one 16-row slab each
 constexpr int kSkThreads = 32 * kSkWarps;
 #ifndef WQ_SK_MIN_M
-#define WQ_SK_MIN_M 5
+#define WQ_SK_MIN_M 2
 #endif
 constexpr int kSkMinM = WQ_SK_MIN_M;  // wq_gemm / wq_linear_set use this kernel for int4 from
-                                      // this M (below it the streaming kernel is faster) ...
+                                      // this M (at M = 1 the streaming GEMV is faster) ...
 constexpr int kSkMaxM = 32;           // ... up to this M (tokens per product)
 constexpr int kSkMaxMats = 256;
 // code groups in flight per thread (cp.async ring of 16 KB slots): six for up to 16 tokens;

@@ -96,7 +96,7 @@ int wq_gemv(const uint16_t* x, const void* codes, const uint16_t* scale,
 
 /* Y[m, n] = fp16( sum_k X[m, k] * w_hat[n, k] ) for M activation rows, 1 <= M <= 2048.
  * M = 1 runs the wq_gemv kernel. Small M streams the weights once and reuses each
- * dequantised weight for every row of X (int4 with 5 <= M <= 32: warp-level tensor-core
+ * dequantised weight for every row of X (int4 with 2 <= M <= 32: warp-level tensor-core
  * MMAs fed from registers); large M dequantises weight tiles into shared memory as fp16
  * tensor-core operands with fp32 accumulators (TKintegers K5, "What is K5?": tiles
  * expanded to fp16 tensor-core operands, fp32 accumulation). */
@@ -120,9 +120,9 @@ typedef struct {
 #define WQ_LINEAR_SET_MAX 256
 
 /* Run `count` independent products of one format as ONE persistent kernel launch per kind
- * of kernel (streaming kernel for M <= 4, skinny-batch kernel for int4 with 5 <= M <= 32,
- * tensor-core GEMM for int4 with larger M -- split into launches of at most 80 matrices --,
- * the generic set kernel otherwise). `descs` is a
+ * of kernel (streaming kernel for M = 1 and for int2 / ternary up to M = 4, skinny-batch
+ * kernel for int4 with 2 <= M <= 32, tensor-core GEMM for int4 with larger M -- split into
+ * launches of at most 80 matrices --, the generic set kernel otherwise). `descs` is a
  * HOST array (read during the call, not kept); the pointers inside are device pointers.
  * Equivalent to count wq_gemm calls, without count launches: at batch 1 a whole decoded
  * token reads every weight once, and per-launch overhead dominates small matrices

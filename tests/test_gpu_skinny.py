@@ -1,4 +1,4 @@
-"""Parity of the skinny-batch int4 GEMM (a few tokens, warp-level MMAs fed from registers)
+"""Parity of the skinny-batch int4 GEMM (M = 2..32 tokens, warp-level MMAs fed from registers)
 with the oracle, through wq_gemm / wq_linear_set.
 
 Covers every token-block count (M up to 8, 16 and 32) and the M at their edges, weight
@@ -20,7 +20,7 @@ from test_gpu_parity import _crafted_weights
 
 pytestmark = pytest.mark.gpu
 
-MS = [5, 7, 8, 9, 15, 16, 17, 24, 31, 32]
+MS = [2, 3, 4, 5, 7, 8, 9, 15, 16, 17, 24, 31, 32]
 SHAPES = [(1, 128), (7, 256), (129, 896), (300, 1024), (333, 4864), (40, 7168)]
 
 
@@ -37,7 +37,7 @@ def test_skinny_gemm_matches_oracle(M, N, K):
     assert_within_tol(f16_np(Y), y_ref, bound, f"skinny M={M} {N}x{K}")
 
 
-@pytest.mark.parametrize("M", [5, 16, 32])
+@pytest.mark.parametrize("M", [2, 5, 16, 32])
 def test_skinny_set_equals_single_calls(M):
     shapes = [(896, 896), (128, 896), (333, 1152), (40, 4864), (513, 256), (256, 128), (1000, 3584)]
     ent, singles = [], []
@@ -56,7 +56,7 @@ def test_skinny_set_equals_single_calls(M):
         assert torch.equal(Y, Ys), (M, N, K)
 
 
-@pytest.mark.parametrize("M", [5, 12, 32])
+@pytest.mark.parametrize("M", [2, 5, 12, 32])
 def test_skinny_special_cases(M):
     N, K = 77, 1024
     W = synth.weights(N, K, 0.02, seed=11)
