@@ -266,6 +266,40 @@ def quantize(W, fmt: str):
 
 
 # --------------------------------------------------------------------------------------
+# Head rescoring.  Whetstone README, feature list (--head-rescore): an fp16 copy of the
+# output projection is kept, and only the logits that decide the token are recomputed
+# from it.  READING: the logits that decide the token are the k largest quantised-head
+# logits (ties to the lower row); each is recomputed as the product of x with the fp16
+# row, and the token is the row with the largest recomputed logit (ties to the lower row).
+# --------------------------------------------------------------------------------------
+
+def topk_rows(y, k: int) -> np.ndarray:
+    """Rows of the k largest values of y (1-D), largest first, equal values by lower row.
+
+    A stable sort on the negated values is the definition written out: numpy's stable
+    argsort keeps equal keys in index order. k is clipped to len(y)."""
+    yd = np.asarray(y, dtype=np.float64)
+    order = np.argsort(-yd, kind="stable")
+    return order[: min(k, len(yd))].astype(np.int64)
+
+
+def rescore(x, w16_rows) -> tuple[np.ndarray, np.ndarray]:
+    """The candidates' logits from the fp16 head: linear() of x with the given fp16 rows.
+
+    Returns (logits, bound), float64, for the acceptance test |l_gpu - l| <= 2e-3 bound."""
+    w = np.asarray(w16_rows).astype(np.float64)
+    return linear(np.asarray(x).reshape(-1), w)
+
+
+def pick_token(rows, logits) -> int:
+    """The row with the largest logit among the candidates; equal logits: the lower row."""
+    rows = np.asarray(rows, dtype=np.int64)
+    lg = np.asarray(logits, dtype=np.float64)
+    best = lg.max()
+    return int(rows[lg == best].min())
+
+
+# --------------------------------------------------------------------------------------
 # Whetstone README, "Measured hardware facts": for a, b in {-1,+1}^K packed as bits
 # {1, 0}, dot(a, b) = K - 2 popcount(a XOR b).
 # --------------------------------------------------------------------------------------

@@ -330,6 +330,45 @@ def test_linear_special_cases():
     assert Y.shape == (3, 5)
 
 
+# ---- head rescoring (Whetstone README feature list, --head-rescore) -------------------
+
+def _topk_brute(y, k):
+    """Repeatedly take the largest remaining value, the lowest row among equals."""
+    left = list(range(len(y)))
+    out = []
+    for _ in range(min(k, len(y))):
+        best = left[0]
+        for i in left[1:]:
+            if y[i] > y[best]:
+                best = i
+        out.append(best)
+        left.remove(best)
+    return out
+
+
+def test_topk_rows_matches_brute_force_with_ties():
+    rng = np.random.default_rng(11)
+    for n, k in ((1, 1), (5, 8), (40, 8), (200, 64), (64, 64)):
+        y = rng.integers(-3, 4, n).astype(np.float16)   # many equal values
+        assert O.topk_rows(y, k).tolist() == _topk_brute([float(v) for v in y], k)
+    y = np.array([1.0, 2.0, 2.0, -0.0, 0.0, 2.0], np.float16)
+    assert O.topk_rows(y, 4).tolist() == [1, 2, 5, 0]
+
+
+def test_rescore_is_exact_sum_and_pick_is_lowest_max():
+    rng = np.random.default_rng(12)
+    K = 256
+    x = rng.integers(-4, 5, K).astype(np.float16)          # small integers: every product
+    rows = rng.integers(-8, 9, (6, K)).astype(np.float16)   # and sum is exact in float64
+    lg, bound = O.rescore(x, rows)
+    for i in range(6):
+        assert lg[i] == sum(int(a) * int(b) for a, b in zip(x, rows[i]))
+        assert bound[i] == sum(abs(int(a) * int(b)) for a, b in zip(x, rows[i]))
+    cand = [40, 7, 19, 3]
+    assert O.pick_token(cand, [1.0, 5.0, 5.0, 2.0]) == 7      # tie: lower row
+    assert O.pick_token(cand, [9.0, 5.0, 5.0, 2.0]) == 40
+
+
 # ---- planted mistakes are caught -----------------------------------------------------
 
 def test_planted_mistakes_are_caught(monkeypatch):
