@@ -234,6 +234,23 @@ def bench_rows(args, pk):
             ms = time_steps(step_am, 200 if not args.quick else 20, 10, 1)
             rows["gemv_argmax_lm_head_int4"] = {"ms": ms, "GBps": nb / ms / 1e6,
                                                 "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"]}
+            # head rescoring: int4 head, top 8 candidates recomputed from an fp16 head copy
+            topk = 8
+            w16 = synth.weights_with_outliers(N, K, wl["sigma"], synth.sub_seed(wl["seed"], 0, 0),
+                                              wl["outlier_frac"], wl["outlier_gain"], device="cuda").half()
+            wsr = torch.empty(wq.wq_rescore_workspace_bytes(N, topk), dtype=torch.uint8, device="cuda")
+            cand = torch.empty(topk, dtype=torch.int32, device="cuda")
+            cl = torch.empty(topk, dtype=torch.float32, device="cuda")
+            tok = torch.empty(1, dtype=torch.int32, device="cuda")
+
+            def step_rs(i, copies=copies):
+                c, s, z = copies[i % len(copies)]
+                wq.wq_gemv_rescore(x, c, s, z, "int4", w16, N, K, topk, y, cand, cl, tok, wsr, wsr.numel())
+            ms = time_steps(step_rs, 200 if not args.quick else 20, 10, 1)
+            rows["gemv_rescore_lm_head_int4"] = {"ms": ms, "GBps": nb / ms / 1e6,
+                                                 "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"],
+                                                 "topk": topk, "launches": 3}
+            del w16
         del copies
         torch.cuda.empty_cache()
     rows.update(bench_batch_sweep(args, pk))

@@ -25,6 +25,7 @@ FMT = {"int4": WQ_INT4, "int2": WQ_INT2, "ternary": WQ_TERNARY}
 WQ_OK, WQ_ERR_ARG, WQ_ERR_SHAPE, WQ_ERR_ALIGN, WQ_ERR_CUDA, WQ_ERR_UNSUPPORTED, WQ_ERR_SCRATCH = range(7)
 WQ_ARGMAX_STATIC_SCRATCH_BYTES = 16384
 WQ_LINEAR_SET_MAX = 256
+WQ_RESCORE_MAX_TOPK = 64
 
 _i64, _p, _i = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
 
@@ -47,6 +48,9 @@ _sig = {
     "wq_argmax_workspace_bytes": (ctypes.c_size_t, []),
     "wq_gemv_argmax": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p, _p, ctypes.c_size_t, _p]),
     "wq_gemv_argmax_static": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p, _p]),
+    "wq_rescore_workspace_bytes": (ctypes.c_size_t, [_i64, _i]),
+    "wq_gemv_rescore": (_i, [_p, _p, _p, _p, _i, _p, _i64, _i64, _i, _p, _p, _p, _p, _p,
+                             ctypes.c_size_t, _p]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -127,6 +131,20 @@ def wq_gemv_argmax_static(x, codes, scale, zero, fmt, N, K, y, argmax, stream=No
     _check(_lib.wq_gemv_argmax_static(_ptr(x), _ptr(codes), _ptr(scale), _ptr(zero), _fmt(fmt),
                                       N, K, _ptr(y), _ptr(argmax), _stream(stream)),
            "wq_gemv_argmax_static")
+
+
+def wq_rescore_workspace_bytes(N, topk) -> int:
+    return _lib.wq_rescore_workspace_bytes(N, topk)
+
+
+def wq_gemv_rescore(x, codes, scale, zero, fmt, w16, N, K, topk, y, cand, cand_logits, token,
+                    workspace, workspace_bytes, stream=None) -> None:
+    """Head rescoring: y (fp16 [N]), cand (int32 [topk]), cand_logits (fp32 [topk]) and
+    token (int32 [1]) are device tensors; w16 is the fp16 head [N, K]."""
+    _check(_lib.wq_gemv_rescore(_ptr(x), _ptr(codes), _ptr(scale), _ptr(zero), _fmt(fmt),
+                                _ptr(w16), N, K, topk, _ptr(y), _ptr(cand), _ptr(cand_logits),
+                                _ptr(token), _ptr(workspace), workspace_bytes, _stream(stream)),
+           "wq_gemv_rescore")
 
 
 def make_linear_set(entries) -> ctypes.Array:

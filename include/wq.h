@@ -173,6 +173,30 @@ int wq_gemv_argmax_static(const uint16_t* x, const void* codes, const uint16_t* 
                           const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* y,
                           int32_t* argmax, void* stream);
 
+/* Largest candidate count of wq_gemv_rescore. */
+#define WQ_RESCORE_MAX_TOPK 64
+
+/* Work-space bytes wq_gemv_rescore needs for N rows and topk candidates (0 if N or topk is
+ * out of range: 1 <= N <= 524288, 1 <= topk <= WQ_RESCORE_MAX_TOPK). */
+size_t wq_rescore_workspace_bytes(int64_t N, int topk);
+
+/* Head rescoring (Whetstone README, feature list: --head-rescore keeps an fp16 copy of the
+ * output projection and recomputes only the logits that decide the token).
+ *   y           = the quantised head's logits, exactly as wq_gemv (fp16 [N]);
+ *   cand[i]     = the rows of the topk largest y, largest first, equal y: lower row first
+ *                 (int32 [topk]; only the first min(topk, N) entries are written);
+ *   cand_logits = fp32 sum over k of x[k] * w16[cand[i], k] (float [topk]), each product exact;
+ *   *token      = the candidate with the largest cand_logits, equal values: the lower row.
+ * w16: the fp16 head, [N, K] row-major, 16-byte aligned (e.g. the fp32 weights rounded to
+ * fp16). workspace: device memory of at least wq_rescore_workspace_bytes(N, topk) bytes,
+ * 8-byte aligned, owned by the caller; no state is kept in it between calls. The other
+ * arguments and requirements are wq_gemv's. All checks run before the first launch; three
+ * launches on `stream` (the GEMV, a per-chunk top-k, one merge-and-recompute CTA). */
+int wq_gemv_rescore(const uint16_t* x, const void* codes, const uint16_t* scale,
+                    const uint16_t* zero, int fmt, const uint16_t* w16, int64_t N, int64_t K,
+                    int topk, uint16_t* y, int32_t* cand, float* cand_logits, int32_t* token,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static string naming a status code. */
 const char* wq_status_str(int status);
 

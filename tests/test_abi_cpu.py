@@ -85,3 +85,25 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert wq._lib.wq_linear_set(arr, 257, 0, S) == wq.WQ_ERR_ARG
     assert wq._lib.wq_linear_set(None, 1, 0, S) == wq.WQ_ERR_ARG
     assert wq.wq_status_str(wq.WQ_ERR_ALIGN).startswith("WQ_ERR_ALIGN")
+
+
+def test_rescore_sizes_and_argument_checks(lib):
+    from bit_weight_quantized_unpack_b200 import wq
+    # one 8-byte key per candidate and 2048-logit chunk
+    assert wq.wq_rescore_workspace_bytes(151936, 8) == 75 * 8 * 8
+    assert wq.wq_rescore_workspace_bytes(1, 1) == 8
+    assert wq.wq_rescore_workspace_bytes(524288, 64) == 256 * 64 * 8
+    assert wq.wq_rescore_workspace_bytes(524289, 8) == 0
+    assert wq.wq_rescore_workspace_bytes(100, 0) == 0
+    assert wq.wq_rescore_workspace_bytes(100, wq.WQ_RESCORE_MAX_TOPK + 1) == 0
+    P = 1 << 20   # a 16-byte aligned fake address: never dereferenced on a rejected call
+    ws = 1 << 16
+    f = wq._lib.wq_gemv_rescore
+    assert f(P, P, P, P, 0, None, 1000, 128, 8, P, P, P, P, P, ws, None) == wq.WQ_ERR_ARG   # no fp16 head
+    assert f(P, P, P, P, 0, P, 1000, 128, 0, P, P, P, P, P, ws, None) == wq.WQ_ERR_ARG      # topk 0
+    assert f(P, P, P, P, 0, P, 1000, 128, 65, P, P, P, P, P, ws, None) == wq.WQ_ERR_ARG     # topk > 64
+    assert f(P, P, P, P, 0, P, 524289, 128, 8, P, P, P, P, P, ws, None) == wq.WQ_ERR_SHAPE  # too many rows
+    assert f(P, P, P, P, 0, P, 1000, 100, 8, P, P, P, P, P, ws, None) == wq.WQ_ERR_SHAPE    # K % 128
+    assert f(P, P, P, P, 0, P, 1000, 128, 8, P, P, P, P, P, 8, None) == wq.WQ_ERR_ARG       # small work space
+    assert f(P, P, P, P, 0, P + 8, 1000, 128, 8, P, P, P, P, P, ws, None) == wq.WQ_ERR_ALIGN
+    assert f(P, P, P, P, 0, P, 1000, 128, 8, P, P, P, P, P + 4, ws, None) == wq.WQ_ERR_ALIGN
