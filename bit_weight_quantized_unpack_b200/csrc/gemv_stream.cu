@@ -707,13 +707,13 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   p.xbuf_bytes = (mt * (max_k / kGroup) * F::XU * 16 + 127) & ~127;
   p.errors = device_error_word();
   if (!p.errors) return 0;
-  // two ring slots per warp; two activation buffers when four CTAs still fit on an SM
-  // (measured best on the 0.5B decode set), else one; then as many CTAs as fit
-  const int ring = W * 2 * (F::SLOT + 8) + F::LUT;
+  // kStreamSlots ring slots per warp; two activation buffers when four CTAs still fit on an
+  // SM (measured best on the 0.5B decode set), else one; then as many CTAs as fit
+  const int ring = W * kStreamSlots * (F::SLOT + 8) + F::LUT;
   const int two = ring + 2 * p.xbuf_bytes, one = ring + p.xbuf_bytes;
   const int bytes = (kStreamSmPool / (two + 1024) >= kStreamMaxCtasPerSm) ? two : one;
   if (bytes > kStreamMaxSmem) return 0;
-  p.slots = 2;
+  p.slots = kStreamSlots;
   p.xbufs = bytes == two ? 2 : 1;
   const int fit = kStreamSmPool / (bytes + 1024);
   p.ctas_per_sm = fit < kStreamMaxCtasPerSm ? fit : kStreamMaxCtasPerSm;

@@ -12,7 +12,14 @@ constexpr int kStreamMaxMats = 256;
 constexpr int kStreamMaxRows = 4;            // rows of X per product (M = 1 .. 4)
 constexpr int kStreamSmPool = 233472;        // shared memory of one SM (228 KB)
 constexpr int kStreamMaxSmem = 232448 - 1024; // dynamic, per CTA (227 KB less room for static)
-constexpr int kStreamSlotCodes = 4096;       // bytes of codes per ring slot (one bulk copy)
+#ifndef WQ_STREAM_SLOT_CODES
+#define WQ_STREAM_SLOT_CODES 4096
+#endif
+#ifndef WQ_STREAM_SLOTS
+#define WQ_STREAM_SLOTS 2
+#endif
+constexpr int kStreamSlotCodes = WQ_STREAM_SLOT_CODES;  // bytes of codes per ring slot (one bulk copy)
+constexpr int kStreamSlots = WQ_STREAM_SLOTS;           // ring slots per warp
 
 // One matrix. Rows are dealt to warps in units of RA rows, RA chosen so that every unit's
 // scales and zeros start on a 16-byte boundary; cost counts bytes of codes + scales + zeros.
