@@ -10,8 +10,9 @@ namespace wq {
 constexpr int kTcMaxBN = 256;   // tokens per tile (MMA N), also the TMEM columns allocated
 constexpr int kTcMaxMats = 80;  // matrices per launch: 80 x 384 B of tensor maps and fields fit
                                 // the 32 KB kernel parameter block
-constexpr int kTcMinM = 5;      // wq_gemm uses the tensor-core path from this M up (int4);
-                                // token rows past M in a 16-row tile are zero-filled by TMA
+constexpr int kTcMinM = 5;      // int4 products from this M up that the skinny-batch kernel
+                                // does not take (M > 32, or its alignment needs unmet) run
+                                // here; token rows past M in a 16-row tile are zero-filled by TMA
 
 // One matrix: tiles [tile_begin, tile_end) of the launch, tiles_m token tiles per
 // 128-row weight tile. Tensor maps first: CUtensorMap needs 64-byte alignment.
