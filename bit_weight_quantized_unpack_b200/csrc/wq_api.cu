@@ -6,7 +6,6 @@
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
-#include "gemv_bulk.cuh"
 #include "gemv_rows.cuh"
 #include "gemv_stream.cuh"
 #include "wq.h"
@@ -51,10 +50,6 @@ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0;
 
 constexpr int64_t kMaxK = (int64_t)1 << 20;
 
-// Which matrix-vector kernel serves batch 1: the register-streaming kernel (gemv.cu) or
-// the bulk-copy-staged one (gemv_bulk.cu). Both compute identical results.
-constexpr bool kUseBulkGemv = false;
-
 int check_shape(int fmt, int64_t N, int64_t K) {
   if (fmt < WQ_INT4 || fmt > WQ_TERNARY) return WQ_ERR_ARG;
   if (N < 1 || N > INT_MAX || K < 128 || K > kMaxK || K % 128 != 0) return WQ_ERR_SHAPE;
@@ -85,32 +80,6 @@ int64_t plan_mat(wq::SetMat& m, int fmt, const void* codes, const uint16_t* scal
   m.lanes_log2 = wq::gemv_lanes_log2(fmt, K);
   const int64_t rows = 32 >> m.lanes_log2;
   return (N + rows - 1) / rows;
-}
-
-// Plan the bulk-staged kernel for entries [0, count) of a set (int4 / int2, batch 1).
-// Returns false if any matrix needs the register-streaming kernel instead.
-bool plan_bulk(wq::BulkParams& p, int fmt, int count, const wq_linear_desc* d) {
-  if (fmt == WQ_TERNARY || count > wq::kBulkMaxMats) return false;
-  const int bits = fmt == WQ_INT4 ? 4 : 2;
-  p.errors = wq::device_error_word();
-  if (!p.errors) return false;
-  p.count = count;
-  int64_t blocks = 0, cost = 0;
-  for (int i = 0; i < count; ++i) {
-    wq::BulkMat& m = p.m[i];
-    if (!wq::bulk_plan_mat(m, bits, d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K))
-      return false;
-    const int64_t nb = (d[i].N + m.rows_per_block - 1) / m.rows_per_block;
-    m.block_begin = (int)blocks;
-    m.cost_begin = cost;
-    blocks += nb;
-    cost += nb * m.block_bytes;
-    if (blocks > INT_MAX) return false;
-    m.block_end = (int)blocks;
-  }
-  p.total_blocks = (int)blocks;
-  p.total_cost = cost;
-  return true;
 }
 
 // Streaming kernel for a set (int4 / int2) with M = 1 .. 4 rows of X: needs 16-byte aligned
@@ -226,11 +195,6 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
       if (done) return r;
     }
   }
-  if (M == 1 && fmt != WQ_TERNARY && kUseBulkGemv) {
-    static thread_local wq::BulkParams bp;
-    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, 1};
-    if (plan_bulk(bp, fmt, 1, &d)) return cuda_status(wq::launch_gemv_bulk(bp, fmt == WQ_INT4 ? 4 : 2, (cudaStream_t)stream));
-  }
   wq::SetParams p;
   p.count = 1;
   const int64_t items = plan_mat(p.m[0], fmt, codes, scale, zero, X, Y, N, K, M);
@@ -324,11 +288,6 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
       r = try_rows(fmt, count, descs, (cudaStream_t)stream, &done);
       if (done) return r;
     }
-  }
-  if (kUseBulkGemv) {
-    static thread_local wq::BulkParams bp;
-    if (plan_bulk(bp, fmt, count, descs))
-      return cuda_status(wq::launch_gemv_bulk(bp, fmt == WQ_INT4 ? 4 : 2, (cudaStream_t)stream));
   }
   for (int i = count; i < wq::kSetMax; ++i) {
     memset(&p.m[i], 0, sizeof(p.m[i]));
