@@ -80,8 +80,11 @@ def f16_from_bits(b) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 # Quantisers.  Whetstone README, "What the weights can actually survive": round-to-nearest
 # at group 128, with one fp16 scale and one fp16 zero per group (0.25 bits/weight of
-# metadata); format table rows int4 g128 (4.25), int2 g128 (2.25), ternary g128 (1.71).
+# metadata); format table rows int4 g128 (4.25), int3 g128 (3.25), int2 g128 (2.25),
+# ternary g128 (1.71).
 # --------------------------------------------------------------------------------------
+
+INT_BITS = {"int4": 4, "int3": 3, "int2": 2}
 
 def quantize_int(W, bits: int):
     """Asymmetric round-to-nearest group-128 quantisation along K to `bits`-bit codes.
@@ -93,12 +96,16 @@ def quantize_int(W, bits: int):
         z  = clamp(rint(-lo / s), 0, Q)          (integer zero point, stored as fp16)
         q  = clamp(rint(w / s) + z, 0, Q)        (rint: ties to even)
     so that w ~ w_hat = (q - z) * s with the stored fp16 s and z.
-    Returns codes uint32 [N, K*bits/32] (code k in word k // (32/bits), bits
-    bits*(k % (32/bits)), little-endian fields), scale and zero as uint16 fp16 bits [N, K/128].
+    Returns codes uint32 [N, K*bits/32] (code k at bits bits*k .. bits*k + bits - 1 of the
+    row's little-endian bit stream, word j holding stream bits 32 j .. 32 j + 31: for 2 and 4
+    bits word k // (32/bits), bits bits*(k % (32/bits)); 3-bit codes may straddle two
+    words), scale and zero as uint16 fp16 bits [N, K/128].
+    READING for int3 (the format table gives only "int3 g128", 3.25 bits/weight): the same
+    quantiser with Q = 7 and the same bit-stream order as int2 / int4.
     """
     W = np.asarray(W)
     N, K = W.shape
-    assert K % GROUP == 0 and bits in (2, 4)
+    assert K % GROUP == 0 and bits in (2, 3, 4)
     G = K // GROUP
     Q = float(2 ** bits - 1)
     w = W.astype(np.float64).reshape(N, G, GROUP)
@@ -112,9 +119,12 @@ def quantize_int(W, bits: int):
 
 
 def pack_int(q, bits: int) -> np.ndarray:
-    """Pack codes [N, K] (< 2^bits) into uint32 words, code k at bit bits*(k % per)."""
+    """Pack codes [N, K] (< 2^bits) into uint32 words, code k at bits bits*k.. of the row's
+    little-endian bit stream (for 2 and 4 bits: word k // per, bit bits*(k % per))."""
     q = np.asarray(q, dtype=np.uint32)
     N, K = q.shape
+    if 32 % bits:
+        return _pack_stream(q, bits)
     per = 32 // bits
     q = q.reshape(N, K // per, per)
     words = np.zeros((N, K // per), dtype=np.uint32)
@@ -123,8 +133,41 @@ def pack_int(q, bits: int) -> np.ndarray:
     return words
 
 
+def _pack_stream(q, bits: int) -> np.ndarray:
+    """Bit-stream packing for code widths that do not divide 32: code k's bit b goes to
+    stream bit bits*k + b, i.e. word (bits*k + b) // 32, bit (bits*k + b) % 32."""
+    N, K = q.shape
+    assert (K * bits) % 32 == 0
+    words = np.zeros((N, K * bits // 32), dtype=np.uint64)
+    for k in range(K):
+        pos = bits * k
+        j, off = divmod(pos, 32)
+        v = q[:, k].astype(np.uint64) << np.uint64(off)        # up to 34 bits
+        words[:, j] |= v & np.uint64(0xFFFFFFFF)
+        if off + bits > 32:
+            words[:, j + 1] |= v >> np.uint64(32)
+    return words.astype(np.uint32)
+
+
+def _unpack_stream(codes, bits: int, K: int) -> np.ndarray:
+    """Inverse of _pack_stream."""
+    codes = np.asarray(codes, dtype=np.uint32).astype(np.uint64)
+    N = codes.shape[0]
+    out = np.empty((N, K), dtype=np.int64)
+    mask = np.uint64(2 ** bits - 1)
+    for k in range(K):
+        j, off = divmod(bits * k, 32)
+        v = codes[:, j] >> np.uint64(off)
+        if off + bits > 32:
+            v |= codes[:, j + 1] << np.uint64(32 - off)
+        out[:, k] = (v & mask).astype(np.int64)
+    return out
+
+
 def unpack_int(codes, bits: int, K: int) -> np.ndarray:
     """Inverse of pack_int: uint32 words [N, K*bits/32] -> codes int64 [N, K]."""
+    if 32 % bits:
+        return _unpack_stream(codes, bits, K)
     codes = np.asarray(codes, dtype=np.uint32)
     N = codes.shape[0]
     per = 32 // bits
@@ -253,7 +296,7 @@ def gemv_packed(x, fmt: str, packed, scale_bits, zero_bits, K: int):
     if fmt == "ternary":
         w_hat = dequant_ternary(packed, scale_bits, K)
     else:
-        w_hat = dequant_int(packed, scale_bits, zero_bits, {"int4": 4, "int2": 2}[fmt], K)
+        w_hat = dequant_int(packed, scale_bits, zero_bits, INT_BITS[fmt], K)
     return linear(x, w_hat)
 
 
@@ -262,7 +305,7 @@ def quantize(W, fmt: str):
     if fmt == "ternary":
         p, s = quantize_ternary(W)
         return p, s, None
-    return quantize_int(W, {"int4": 4, "int2": 2}[fmt])
+    return quantize_int(W, INT_BITS[fmt])
 
 
 # --------------------------------------------------------------------------------------
@@ -344,5 +387,4 @@ def stored_bits_per_weight(fmt: str) -> float:
     """Bits per weight of this layout as stored: codes + fp16 metadata per 128 weights."""
     if fmt == "ternary":
         return (TERNARY_GROUP_BYTES * 8 + 16) / GROUP
-    b = {"int4": 4, "int2": 2}[fmt]
-    return b + 32 / GROUP
+    return INT_BITS[fmt] + 32 / GROUP

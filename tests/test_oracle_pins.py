@@ -71,8 +71,9 @@ def test_stored_layout_bits_per_weight():
     assert O.stored_bits_per_weight("int2") == 2.25
     # 26 bytes + one fp16 scale per 128 trits, against the information content 1.71
     assert O.stored_bits_per_weight("ternary") == 1.75
+    assert O.stored_bits_per_weight("int3") == 3.25       # format table row "int3 g128"
     W = np.random.default_rng(0).normal(0, 0.02, (8, 256)).astype(np.float32)
-    for fmt, bits in (("int4", 4.25), ("int2", 2.25), ("ternary", 1.75)):
+    for fmt, bits in (("int4", 4.25), ("int3", 3.25), ("int2", 2.25), ("ternary", 1.75)):
         p, s, z = O.quantize(W, fmt)
         nbytes = p.nbytes + s.nbytes + (0 if z is None else z.nbytes)
         assert nbytes * 8 / W.size == bits
@@ -167,7 +168,7 @@ def test_constant_and_nonnegative_groups():
 
 def test_rtn_is_nearest_code_within_range():
     rng = np.random.default_rng(2)
-    for bits in (4, 2):
+    for bits in (4, 3, 2):
         Q = 2 ** bits - 1
         W = rng.normal(0, 0.02, (16, 512)).astype(np.float32)
         codes, sb, zb = O.quantize_int(W, bits)
@@ -328,6 +329,49 @@ def test_linear_special_cases():
         ym, _ = O.gemv_packed(X[m], "int4", codes, sb, zb, 256)
         assert np.allclose(Y[m], ym, rtol=1e-14, atol=0)
     assert Y.shape == (3, 5)
+
+
+# ---- int3 g128: 3-bit codes in the row's little-endian bit stream ----------------------
+
+# codes 0, 1, ..., 7 repeated: eight codes are the 24-bit number 0o76543210 = 0xFAC688, so
+# the little-endian byte stream is 88 C6 FA repeated, and the first three words are these
+INT3_RAMP_WORDS = [0x88FAC688, 0xC688FAC6, 0xFAC688FA]
+
+
+def test_int3_bit_stream_packing():
+    q = (np.arange(256) % 8).reshape(1, 256)
+    words = O.pack_int(q, 3)
+    assert words.shape == (1, 24)
+    assert words[0, :3].tolist() == INT3_RAMP_WORDS
+    assert bytes(words.view(np.uint8)) == bytes([0x88, 0xC6, 0xFA]) * 32
+    # random codes against the stream written as one integer, and the round trip
+    rng = np.random.default_rng(21)
+    q = rng.integers(0, 8, (3, 384))
+    w = O.pack_int(q, 3)
+    for n in range(3):
+        big = sum(int(v) << (3 * k) for k, v in enumerate(q[n]))
+        assert w[n].tolist() == [(big >> (32 * j)) & 0xFFFFFFFF for j in range(w.shape[1])]
+    assert np.array_equal(O.unpack_int(w, 3, 384), q)
+
+
+def test_int3_ramp_codes_and_dequant_definition():
+    j = np.arange(256)
+    ramp = (-1 + 0.25 * (j % 8)).reshape(1, 256).astype(np.float32)   # 8 levels, step 0.25
+    codes, sb, zb = O.quantize_int(ramp, 3)
+    assert codes[0, :3].tolist() == INT3_RAMP_WORDS
+    assert np.all(O.f16_from_bits(sb) == 0.25) and np.all(O.f16_from_bits(zb) == 4.0)
+    # w_hat from the codes read back bit by bit, against the oracle's dequantiser
+    rng = np.random.default_rng(22)
+    W = rng.normal(0, 0.02, (3, 384)).astype(np.float32)
+    c, s, z = O.quantize(W, "int3")
+    w_hat = O.dequant_int(c, s, z, 3, 384)
+    for n in range(3):
+        big = sum(int(v) << (32 * i) for i, v in enumerate(c[n]))
+        for k in range(0, 384, 7):
+            q = (big >> (3 * k)) & 7
+            sk = float(O.f16_from_bits(s[n, k // 128]))
+            zk = float(O.f16_from_bits(z[n, k // 128]))
+            assert w_hat[n, k] == (q - zk) * sk
 
 
 # ---- head rescoring (Whetstone README feature list, --head-rescore) -------------------
