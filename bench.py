@@ -193,7 +193,7 @@ def bench_rows(args, pk):
     N, K = 151936, 896
     wl = workloads.WORKLOADS[2]
     # lm_head alone, each format; 4+ rotating copies so the working set exceeds L2
-    for fmt in ("int4", "int2", "ternary"):
+    for fmt in ("int4", "int3", "int2", "ternary"):
         copies = []
         for cidx in range(6 if fmt != "int4" else 4):
             W = synth.weights_with_outliers(N, K, wl["sigma"], synth.sub_seed(wl["seed"] + cidx, 0, 0),

@@ -34,6 +34,8 @@ using SetParams = SetParamsT<kSetMax>;
 
 int gemv_lanes_log2(int fmt, int64_t K);
 cudaError_t launch_gemv_set(const SetParams& p, int fmt, int max_m, cudaStream_t stream);
+// int3 products of a set (one warp per output row, items = rows): gemv_int3.cu
+cudaError_t launch_gemv_int3(const SetParams& p, cudaStream_t stream);
 cudaError_t launch_quantize(const float* W, int64_t N, int64_t K, int fmt, void* codes,
                             uint16_t* scale, uint16_t* zero, cudaStream_t stream);
 

@@ -1,4 +1,4 @@
-// Group-128 quantisers (int4 / int2 asymmetric round-to-nearest, ternary absmean).
+// Group-128 quantisers (int4 / int3 / int2 asymmetric round-to-nearest, ternary absmean).
 //
 // Whetstone README, "What the weights can actually survive": round-to-nearest with group
 // 128 and one fp16 scale plus one fp16 zero per group (format table rows "int4 g128",
@@ -57,7 +57,20 @@ __global__ void __launch_bounds__(256) quantize_int_kernel(const float* __restri
     const double q = fmin(fmax(rint((double)wv[i] / s) + z, 0.0), Q);
     packed |= (uint32_t)q << (BITS * i);
   }
-  if (BITS == 4) {
+  if (BITS == 3) {
+    // lane l holds codes 4l..4l+3: bits 12l..12l+11 of the group's 384-bit stream (12
+    // words); a lane whose 12 bits cross a word boundary contributes to two words
+    const int off = (12 * lane) & 31, w0 = (12 * lane) >> 5;
+    const uint32_t lo = packed << off, hi = off > 20 ? packed >> (32 - off) : 0u;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < 12; ++j) {
+      const uint32_t part = (w0 == j ? lo : 0u) | (w0 + 1 == j ? hi : 0u);
+      const uint32_t word = __reduce_or_sync(0xffffffffu, part);
+      if (lane == j) mine = word;
+    }
+    if (lane < 12) codes[n * (3 * K / 32) + g * 12 + lane] = mine;
+  } else if (BITS == 4) {
     // lanes 2j and 2j+1 hold codes 8j..8j+3 and 8j+4..8j+7 of word j
     packed <<= 16 * (lane & 1);
     packed |= __shfl_xor_sync(0xffffffffu, packed, 1);
@@ -129,6 +142,9 @@ cudaError_t launch_quantize(const float* W, int64_t N, int64_t K, int fmt, void*
                                                                  zero);
   else if (fmt == 1)
     quantize_int_kernel<2><<<(unsigned)blocks, 256, 0, stream>>>(W, N, K, (uint32_t*)codes, scale,
+                                                                 zero);
+  else if (fmt == 3)
+    quantize_int_kernel<3><<<(unsigned)blocks, 256, 0, stream>>>(W, N, K, (uint32_t*)codes, scale,
                                                                  zero);
   else
     quantize_ternary_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, N, K, (uint8_t*)codes, scale);

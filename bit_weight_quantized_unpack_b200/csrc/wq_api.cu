@@ -51,7 +51,7 @@ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0;
 constexpr int64_t kMaxK = (int64_t)1 << 20;
 
 int check_shape(int fmt, int64_t N, int64_t K) {
-  if (fmt < WQ_INT4 || fmt > WQ_TERNARY) return WQ_ERR_ARG;
+  if (fmt < WQ_INT4 || fmt > WQ_INT3) return WQ_ERR_ARG;
   if (N < 1 || N > INT_MAX || K < 128 || K > kMaxK || K % 128 != 0) return WQ_ERR_SHAPE;
   return WQ_OK;
 }
@@ -98,6 +98,33 @@ int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStrea
   return cuda_status(wq::launch_gemv_stream(sp, bits, (int)M, smem, stream));
 }
 
+// int3 set: one warp per output row (any M).
+int launch_int3(const wq_linear_desc* d, int count, cudaStream_t stream) {
+  static thread_local wq::SetParams p;
+  int64_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    wq::SetMat& m = p.m[i];
+    memset(&m, 0, sizeof(m));
+    m.codes = d[i].codes;
+    m.scale = d[i].scale;
+    m.zero = d[i].zero;
+    m.x = d[i].x;
+    m.y = d[i].y;
+    m.N = (int)d[i].N;
+    m.K = (int)d[i].K;
+    m.M = (int)d[i].M;
+    m.ldx = (int)d[i].K;
+    m.ldy = (int)d[i].N;
+    m.item_begin = (int)total;
+    total += d[i].N;
+    if (total > INT_MAX) return WQ_ERR_SHAPE;
+    m.item_end = (int)total;
+  }
+  p.count = count;
+  p.total_items = (int)total;
+  return cuda_status(wq::launch_gemv_int3(p, stream));
+}
+
 // Skinny-batch GEMM for an int4 set with kSkMinM <= M <= kSkMaxM: needs 16-byte aligned
 // codes and activations.
 int try_skinny(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStream_t stream, bool* done) {
@@ -137,6 +164,7 @@ size_t wq_codes_bytes(int fmt, int64_t N, int64_t K) {
   if (check_shape(fmt, N, K) != WQ_OK) return 0;
   if (fmt == WQ_INT4) return (size_t)(N * K / 2);
   if (fmt == WQ_INT2) return (size_t)(N * K / 4);
+  if (fmt == WQ_INT3) return (size_t)(N * K * 3 / 8);
   return (size_t)(N * 26 * (K / 128));
 }
 
@@ -165,6 +193,10 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
   if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
   if (!aligned(X, 16) || !aligned(Y, 2)) return WQ_ERR_ALIGN;
   if ((st = check_device()) != WQ_OK) return st;
+  if (fmt == WQ_INT3) {
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, M};
+    return launch_int3(&d, 1, (cudaStream_t)stream);
+  }
   {
     const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, M};
     bool done = false;
@@ -211,7 +243,7 @@ int wq_gemv(const uint16_t* x, const void* codes, const uint16_t* scale, const u
 
 int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream) {
   if (!descs || count < 1 || count > WQ_LINEAR_SET_MAX) return WQ_ERR_ARG;
-  if (fmt < WQ_INT4 || fmt > WQ_TERNARY) return WQ_ERR_ARG;
+  if (fmt < WQ_INT4 || fmt > WQ_INT3) return WQ_ERR_ARG;
   static_assert(WQ_LINEAR_SET_MAX == wq::kSetMax, "set size");
   static thread_local wq::SetParams p;
   p.count = count;
@@ -234,6 +266,7 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   }
   int st0 = check_device();
   if (st0 != WQ_OK) return st0;
+  if (fmt == WQ_INT3) return launch_int3(descs, count, (cudaStream_t)stream);
   {
     bool done = false;
     const int r = try_skinny(fmt, count, descs, M, (cudaStream_t)stream, &done);
@@ -312,7 +345,7 @@ int wq_gemv_argmax(const uint16_t* x, const void* codes, const uint16_t* scale, 
                    void* stream) {
   int st = check_shape(fmt, N, K);
   if (st != WQ_OK) return st;
-  if (fmt == WQ_TERNARY || !x || !argmax || !workspace) return WQ_ERR_ARG;
+  if (fmt == WQ_TERNARY || fmt == WQ_INT3 || !x || !argmax || !workspace) return WQ_ERR_ARG;
   if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
   if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scale, 16) || !aligned(zero, 16) ||
       !aligned(workspace, 16) || (y && !aligned(y, 2)) || !aligned(argmax, 4))

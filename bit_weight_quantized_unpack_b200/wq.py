@@ -20,8 +20,8 @@ if not os.path.exists(_LIB_PATH):
                       "`python -m bit_weight_quantized_unpack_b200.build`")
 _lib = ctypes.CDLL(_LIB_PATH)
 
-WQ_INT4, WQ_INT2, WQ_TERNARY = 0, 1, 2
-FMT = {"int4": WQ_INT4, "int2": WQ_INT2, "ternary": WQ_TERNARY}
+WQ_INT4, WQ_INT2, WQ_TERNARY, WQ_INT3 = 0, 1, 2, 3
+FMT = {"int4": WQ_INT4, "int2": WQ_INT2, "ternary": WQ_TERNARY, "int3": WQ_INT3}
 WQ_OK, WQ_ERR_ARG, WQ_ERR_SHAPE, WQ_ERR_ALIGN, WQ_ERR_CUDA, WQ_ERR_UNSUPPORTED, WQ_ERR_SCRATCH = range(7)
 WQ_ARGMAX_STATIC_SCRATCH_BYTES = 16384
 WQ_LINEAR_SET_MAX = 256

@@ -4,11 +4,11 @@
  *
  * What it computes.  A linear layer y = x . W^T whose weight W [N, K] (N output rows, K
  * along the reduction) is stored quantised in groups of 128 consecutive k of one row:
- *   - WQ_INT4 / WQ_INT2: asymmetric round-to-nearest b-bit codes q in [0, 2^b - 1] with
- *     one fp16 scale s and one fp16 integer zero point z per group, w_hat = (q - z) * s
- *     (Whetstone README, "What the weights can actually survive": round-to-nearest,
- *     group 128, fp16 scale and zero per group; format table rows "int4 g128" 4.25 and
- *     "int2 g128" 2.25 bits/weight);
+ *   - WQ_INT4 / WQ_INT3 / WQ_INT2: asymmetric round-to-nearest b-bit codes q in
+ *     [0, 2^b - 1] with one fp16 scale s and one fp16 integer zero point z per group,
+ *     w_hat = (q - z) * s (Whetstone README, "What the weights can actually survive":
+ *     round-to-nearest, group 128, fp16 scale and zero per group; format table rows
+ *     "int4 g128" 4.25, "int3 g128" 3.25 and "int2 g128" 2.25 bits/weight);
  *   - WQ_TERNARY: trits t in {-1, 0, +1} with one fp16 absmean scale per group,
  *     w_hat = t * s, five trits per byte in base 3 (format table row "ternary g128";
  *     TKintegers K5, "What is K5?": five balanced-ternary digits make a one-byte code).
@@ -30,6 +30,10 @@
  * Layouts (all row-major, rows contiguous; G = K / 128):
  *   int4 codes   uint32 [N, K/8]    code k in word k/8,  bits 4*(k%8)..4*(k%8)+3
  *   int2 codes   uint32 [N, K/16]   code k in word k/16, bits 2*(k%16)..2*(k%16)+1
+ *   int3 codes   uint32 [N, 3K/32]  code k at bits 3k..3k+2 of the row's little-endian
+ *                                   bit stream (word j = stream bits 32j..32j+31; codes
+ *                                   10 and 21 of every 32 straddle two words; a group is
+ *                                   12 words)
  *   ternary      uint8  [N, 26*G]   group g of a row at bytes 26g..26g+25; byte j of a
  *                                   group = sum_{i<5} (t_{5j+i} + 1) * 3^i; byte 25 holds
  *                                   trits 125..127 and two pad trits 0 (digit 1); every
@@ -61,7 +65,7 @@
 extern "C" {
 #endif
 
-typedef enum { WQ_INT4 = 0, WQ_INT2 = 1, WQ_TERNARY = 2 } wq_fmt;
+typedef enum { WQ_INT4 = 0, WQ_INT2 = 1, WQ_TERNARY = 2, WQ_INT3 = 3 } wq_fmt;
 
 typedef enum {
   WQ_OK = 0,
@@ -74,7 +78,7 @@ typedef enum {
 } wq_status;
 
 /* Bytes of packed codes for an [N, K] weight in format fmt (0 on invalid arguments):
- * int4 N*K/2, int2 N*K/4, ternary N*26*(K/128). */
+ * int4 N*K/2, int3 N*K*3/8, int2 N*K/4, ternary N*26*(K/128). */
 size_t wq_codes_bytes(int fmt, int64_t N, int64_t K);
 
 /* Number of fp16 entries of the scale array (and of the zero array): N * K / 128. */

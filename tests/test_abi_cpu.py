@@ -45,14 +45,15 @@ def test_sizes(lib):
     assert lib.wq_codes_bytes(0, 151936, 896) == 151936 * 448
     assert lib.wq_codes_bytes(1, 151936, 896) == 151936 * 224
     assert lib.wq_codes_bytes(2, 151936, 896) == 151936 * 182
+    assert lib.wq_codes_bytes(3, 151936, 896) == 151936 * 336     # int3: 3 bits per code
     assert lib.wq_meta_count(151936, 896) == 151936 * 7
-    # stored bits per weight of the layout: 4.25, 2.25, 1.75
-    for fmt, bpw in ((0, 4.25), (1, 2.25), (2, 1.75)):
+    # stored bits per weight of the layout: 4.25, 2.25, 1.75, 3.25
+    for fmt, bpw in ((0, 4.25), (1, 2.25), (2, 1.75), (3, 3.25)):
         meta_arrays = 1 if fmt == 2 else 2          # scale (+ zero), fp16 each
         tot = lib.wq_codes_bytes(fmt, 64, 1024) + 2 * meta_arrays * lib.wq_meta_count(64, 1024)
         assert tot * 8 / (64 * 1024) == bpw
     assert lib.wq_codes_bytes(0, 4, 100) == 0      # K not a multiple of 128
-    assert lib.wq_codes_bytes(3, 4, 128) == 0      # unknown format
+    assert lib.wq_codes_bytes(4, 4, 128) == 0      # unknown format
     assert lib.wq_codes_bytes(0, 0, 128) == 0
 
 
