@@ -73,7 +73,7 @@ typedef enum {
   WQ_ERR_SHAPE = 2,        /* N, K or M outside the supported range, K % 128 != 0 */
   WQ_ERR_ALIGN = 3,        /* a pointer is not aligned as required above */
   WQ_ERR_CUDA = 4,         /* a CUDA call or launch failed (see wq_last_cuda_error) */
-  WQ_ERR_UNSUPPORTED = 5,  /* valid request this build cannot serve (e.g. no sm_100 GPU) */
+  WQ_ERR_UNSUPPORTED = 5,  /* valid request the library cannot serve here (e.g. no sm_100 GPU) */
   WQ_ERR_SCRATCH = 6       /* needs more scratch than the library's static array holds */
 } wq_status;
 
