@@ -442,3 +442,21 @@ def test_planted_mistakes_are_caught(monkeypatch):
     # (d) identity with a wrong factor
     assert any((K - bin(a ^ b).count("1")) != O.pm1_dot_popcount(a, b, K)
                for K in (3,) for a in range(8) for b in range(8))
+
+    # (e) int3 packed ten codes per word, without crossing word boundaries (2 bits wasted)
+    def pack_no_cross(q):
+        N, K = q.shape
+        nw = -(-K // 10)
+        words = np.zeros((N, nw), dtype=np.uint64)
+        for k in range(K):
+            words[:, k // 10] |= q[:, k].astype(np.uint64) << np.uint64(3 * (k % 10))
+        return words.astype(np.uint32)
+    q = (np.arange(256) % 8).reshape(1, 256)
+    assert pack_no_cross(q)[0, :3].tolist() != INT3_RAMP_WORDS
+
+    # (f) top-k with equal values taken from the higher row first
+    def topk_high(y, k):
+        yd = np.asarray(y, dtype=np.float64)
+        return np.lexsort((-np.arange(len(yd)), -yd))[:k].tolist()   # value, then row, descending
+    y = np.array([1.0, 2.0, 2.0, -0.0, 0.0, 2.0], np.float16)
+    assert topk_high(y, 4) != _topk_brute([float(v) for v in y], 4)
