@@ -44,6 +44,7 @@
 
 #include "common.cuh"
 #include "gemm_skinny.cuh"
+#include "host_util.cuh"
 
 namespace wq {
 
@@ -452,20 +453,11 @@ int skinny_plan(SkParams& p, int count, const SkDesc* d, int M) {
 
 template <int TB>
 static cudaError_t launch_tb(const SkParams& p, int smem, cudaStream_t stream) {
-  static int attr_done[64];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = ensure_smem_limit(gemm_skinny_kernel<TB, kSkMaxMats>, kSkSmemMax, attr_done);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
-    e = cudaFuncSetAttribute(gemm_skinny_kernel<TB, kSkMaxMats>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSkSmemMax);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = 1;
-  }
-  int sms = 0;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  if (sms == 0) return cudaErrorInvalidDevice;
   const int grid = p.total_slabs < sms ? p.total_slabs : sms;  // one CTA per SM
   gemm_skinny_kernel<TB, kSkMaxMats><<<grid, kSkThreads, smem, stream>>>(p);
   return cudaGetLastError();

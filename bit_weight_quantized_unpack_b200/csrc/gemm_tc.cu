@@ -9,23 +9,30 @@
 //     D[n, m] = sum_k w_hat[n0 + n, k] * X[m0 + m, k]      (n < 128, m < BN)
 // and every dequantised weight is reused by all BN tokens of the tile.
 //
-// Per 64-wide k-block (one stage of a 4-stage ring):
-//   - warp 0 (one lane): TMA loads the X tile [BN x 64] fp16 (128-byte swizzle) and the
-//     packed codes [128 rows x 32 bytes], both completing on full[s];
-//   - warps 4-11 (256 threads, two per weight row): dequantise the codes into fp16
-//     (q - z) * s and store them into A[s] in the 128-byte-swizzled K-major layout the
-//     tensor core reads, fence the async proxy, arrive on a_ready[s];
-//   - warp 1 (one lane): waits full[s] and a_ready[s], issues four m128 x nBN x k16 MMAs,
-//     and commits them to empty[s], which frees the stage for the next TMA round.
-// After the last k-block the MMA lane commits to tmem_full; warps 4-11 then read the
-// accumulators (tcgen05.ld) and store fp16 Y[m, n] (one warp store covers 32 consecutive n).
-//
+// Warp roles (one persistent CTA of 16 warps per SM; tiles dealt to CTAs round robin), per
+// 64-wide k-block:
+//   - warp 4 (one lane): TMA loads the activation tile [bn x 64] fp16 (128-byte swizzle) into
+//     an XSTAGES-deep ring, completing on xfull[s]; it waits xempty[s] before reusing a stage;
+//   - warps 8-15 (two teams of four warps, one weight row per thread, the teams taking
+//     alternate k-blocks): copy their rows' packed codes with per-thread cp.async into a
+//     CRING-deep ring, dequantise them into fp16 (q - z) * s, store them into the A stage
+//     in the 128-byte-swizzled K-major layout the tensor core reads, fence the async proxy
+//     and arrive on aready[a] (ASTAGES-deep ring, freed through aempty[a]);
+//   - warp 5 (one lane): allocates the tensor memory; per k-block waits xfull[s] and
+//     aready[a], issues four m128 x n(bn) x k16 tcgen05 MMAs into the tile's accumulator (two
+//     accumulators of 256 columns, alternating tiles) and commits them to xempty[s] and
+//     aempty[a]; after a tile's last k-block it commits to tfull[b];
+//   - warps 0-3 (epilogue, 32 weight rows each): wait tfull[b], read the accumulator with
+//     tcgen05.ld, and store fp16 Y[m, n], through a TMA tensor store of 32 x 32 blocks staged
+//     in shared memory when Y's layout allows, else with plain stores; then arrive on
+//     tempty[b] so that the MMA lane can reuse that accumulator.
 // Every mbarrier wait is bounded; a wait that gives up sets kErrTimeout in the library's
 // device error word, and the CTA drains its own TMA loads, frees its TMEM and exits.
 #include <cuda.h>
 
 #include "common.cuh"
 #include "gemm_tc.cuh"
+#include "host_util.cuh"
 #include "tc_ptx.cuh"
 
 namespace wq {
@@ -467,19 +474,12 @@ int tc_bn_for(int M) {
 
 template <int CAP>
 static cudaError_t launch_cap(const TcParamsT<CAP>& p, cudaStream_t stream) {
-  static bool attr = false;
+  static std::atomic<uint64_t> attr{0};
   const int smem = SMEM_USED + 1024;  // + alignment slack
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_int4_kernel<CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
+  cudaError_t e = ensure_smem_limit(gemm_tc_int4_kernel<CAP>, smem, attr);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  if (sms == 0) return cudaErrorInvalidDevice;
   const int grid = p.total_tiles < sms ? p.total_tiles : sms;
   gemm_tc_int4_kernel<CAP><<<grid, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
@@ -498,15 +498,17 @@ cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream) {
 }
 
 unsigned int* device_error_word() {
-  static unsigned int* addr[64];
+  static std::atomic<unsigned int*> addr[kMaxDevices];  // threads racing on a first call store the same value
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  unsigned int* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_errors) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<unsigned int*>(p);
+    a = static_cast<unsigned int*>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
-  return addr[dev];
+  return a;
 }
 
 cudaError_t read_device_errors(unsigned int* flags, bool clear, cudaStream_t stream) {

@@ -23,6 +23,7 @@
 // grid, so consecutive warps of a CTA work on neighbouring rows of the same matrix.
 #include "common.cuh"
 #include "gemv.cuh"
+#include "host_util.cuh"
 
 namespace wq {
 
@@ -266,12 +267,7 @@ int gemv_lanes_log2(int fmt, int64_t K) {
 }
 
 static int grid_for(const void* kernel, int total_items) {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 1;
   int per_sm = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kGemvThreads, 0);
   if (per_sm < 1) per_sm = 1;

@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "gemv.cuh"
+#include "host_util.cuh"
 
 namespace wq {
 
@@ -104,11 +105,8 @@ __global__ void __launch_bounds__(kInt3Threads) gemv_int3_set_kernel(const __gri
 
 cudaError_t launch_gemv_int3(const SetParams& p, cudaStream_t stream) {
   if (p.total_items < 1) return cudaErrorInvalidValue;
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  if (sms == 0) return cudaErrorInvalidDevice;
   const int wpb = kInt3Threads / 32;
   const int64_t want = ((int64_t)p.total_items + wpb - 1) / wpb;
   const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);

@@ -19,6 +19,7 @@
 // binary32 adds, the multiply by the group scale and the final fp16 store round.
 #include "common.cuh"
 #include "gemv_rows.cuh"
+#include "host_util.cuh"
 
 namespace wq {
 
@@ -265,18 +266,11 @@ bool rows_plan(RowParams& p, int bits, int count, const RowMatDesc* d, int* max_
 template <int BITS, int XM, int CAP>
 static cudaError_t launch_cap(const RowParamsT<CAP>& p, int max_k, cudaStream_t stream) {
   const int smem = kRowsStages * (kGroup * BITS / 8) * THREADS + max_k * (XM == 0 ? 4 : 2);
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel<BITS, XM, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowsMaxSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(gemv_rows_kernel<BITS, XM, CAP>, kRowsMaxSmem, configured);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  if (sms == 0) return cudaErrorInvalidDevice;
   gemv_rows_kernel<BITS, XM, CAP><<<WQ_ROWS_MIN_BLOCKS * sms, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
 }

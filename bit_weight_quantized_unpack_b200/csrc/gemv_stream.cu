@@ -34,6 +34,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_stream.cuh"
+#include "host_util.cuh"
 #include "tc_ptx.cuh"
 
 namespace wq {
@@ -212,6 +213,13 @@ __device__ __forceinline__ void cell_dot_ternary(uint32_t cell, uint32_t xg, uin
   for (int m = 0; m < MT; ++m) out[m] = a[m][0] + a[m][1];
 }
 
+// Wait for an mbarrier phase, giving up after max_polls polls (false).
+__device__ __forceinline__ bool mbar_wait_n(uint32_t bar, uint32_t parity, uint32_t max_polls) {
+  for (uint32_t i = 0; i < max_polls; ++i)
+    if (tc::mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -287,7 +295,8 @@ struct Prod {
 template <int BITS, int MT, bool AM, class Issue>
 __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint32_t xb, uint32_t lut, uint32_t ring,
                                         uint32_t bars, int slots, int& cslot, uint32_t& cphase, int& consumed,
-                                        bool& dead, Issue& issue, int lane, float& bv, int& bi) {
+                                        bool& dead, int& dead_at, uint32_t max_polls, Issue& issue, int lane,
+                                        float& bv, int& bi) {
   using F = Fmt<BITS>;
   const int G = M.K / kGroup;
   const int ncells = seg.groups;
@@ -320,8 +329,11 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
   for (int k = 0; k < nslots; ++k) {
     const uint32_t slot = ring + cslot * F::SLOT;
     if (!dead) {
-      const bool ok = tc::mbar_wait(bars + 8 * cslot, cphase);
-      if (!__all_sync(0xffffffffu, ok)) dead = true;
+      const bool ok = mbar_wait_n(bars + 8 * cslot, cphase, max_polls);
+      if (!__all_sync(0xffffffffu, ok)) {
+        dead = true;
+        dead_at = consumed;  // the copy this wait was for never completed
+      }
     }
     if (F::TRN && crem && k == nslots - 1) {
       const int cl = (int)(seg.bytes & ~(int64_t)15) - k * F::SC;  // slot offset of the tail
@@ -474,8 +486,10 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
   Prod pd;
   pd.cleft = 0;
   pd.pm = mfirst - 1;
-  int issued = 0, consumed = 0;
+  int issued = 0, consumed = 0, dead_at = -1;
   bool dead = false;  // a bounded wait gave up: stop computing, drain, report
+  // failure-detection test hook: CTA 0's warp 0 never fills its first ring slot
+  const bool skip_first = P.skip_first_copy && blockIdx.x == 0 && w == 0;
   auto issue = [&](int slot) {
     while (pd.cleft == 0) {  // next non-empty segment of this warp
       if (++pd.pm >= P.count) return;
@@ -503,11 +517,13 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     // end of a matrix, is loaded by the consumer lanes
     const uint32_t mb = 2u * (uint32_t)(gc & ~7);
     const uint32_t cbb = (uint32_t)cb & ~15u;
-    if (lane == 0) tc::mbar_arrive_expect_tx(bar, cbb + (F::TRN ? 1 : 2) * mb);
-    if (lane == 0 || (lane < (F::TRN ? 2 : 3) && mb)) {
-      const void* src = lane == 0 ? (const void*)pd.c : lane == 1 ? (const void*)pd.s : (const void*)pd.z;
-      const uint32_t d = lane == 0 ? dst : dst + F::SC + (lane - 1) * F::META;
-      bulk_g2s(d, src, lane == 0 ? cbb : mb, bar);
+    if (!(skip_first && issued == 0)) {
+      if (lane == 0) tc::mbar_arrive_expect_tx(bar, cbb + (F::TRN ? 1 : 2) * mb);
+      if (lane == 0 || (lane < (F::TRN ? 2 : 3) && mb)) {
+        const void* src = lane == 0 ? (const void*)pd.c : lane == 1 ? (const void*)pd.s : (const void*)pd.z;
+        const uint32_t d = lane == 0 ? dst : dst + F::SC + (lane - 1) * F::META;
+        bulk_g2s(d, src, lane == 0 ? cbb : mb, bar);
+      }
     }
     pd.c += cb;
     pd.s += gc;
@@ -597,7 +613,8 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     cta_units(M, lo, hi, b0, b1);
     const Seg seg = warp_seg<BITS>(M, b0, b1, w);
     if (seg.rows > 0)
-      consume<BITS, MT, AM>(seg, M, xb, lut, ring, bars, slots, cslot, cphase, consumed, dead, issue, lane, am_v,
+      consume<BITS, MT, AM>(seg, M, xb, lut, ring, bars, slots, cslot, cphase, consumed, dead, dead_at, P.max_polls,
+                            issue, lane, am_v,
                             am_i);
   }
 
@@ -651,10 +668,13 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
   }
 
   // ---- error path: report, then wait (bounded) for copies still landing in this CTA
-  if (__any_sync(0xffffffffu, dead)) {
+  // (dead is warp-uniform); every copy issued after the wait that gave up is waited for, with
+  // the same bound, so that none is still landing in this CTA's shared memory when it exits
+  if (dead) {
     if (lane == 0) {
       atomicOr(P.errors, tc::kErrTimeout);
-      for (int j = consumed; j < issued; ++j) tc::mbar_wait(bars + 8 * (j % slots), (uint32_t)((j / slots) & 1));
+      for (int j = dead_at + 1; j < issued; ++j)
+        mbar_wait_n(bars + 8 * (j % slots), (uint32_t)((j / slots) & 1), P.max_polls);
     }
     __syncwarp();
   }
@@ -707,6 +727,8 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   p.xbuf_bytes = (mt * (max_k / kGroup) * F::XU * 16 + 127) & ~127;
   p.errors = device_error_word();
   if (!p.errors) return 0;
+  p.max_polls = tc::kMaxPolls;
+  p.skip_first_copy = 0;
   // kStreamSlots ring slots per warp; two activation buffers when four CTAs still fit on an
   // SM (measured best on the 0.5B decode set), else one; then as many CTAs as fit
   const int ring = W * kStreamSlots * (F::SLOT + 8) + F::LUT;
@@ -720,26 +742,14 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   return bytes;
 }
 
-int sm_count() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
-  return sms;
-}
-
 template <int BITS, int MT, int CAP, bool AM = false>
 cudaError_t launch_cap(const StreamParamsT<CAP>& p, int smem, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<BITS, MT, CAP, AM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kStreamMaxSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  gemv_stream_kernel<BITS, MT, CAP, AM><<<p.ctas_per_sm * sm_count(), T, smem, stream>>>(p);
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = ensure_smem_limit(gemv_stream_kernel<BITS, MT, CAP, AM>, kStreamMaxSmem, configured);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  if (sms == 0) return cudaErrorInvalidDevice;
+  gemv_stream_kernel<BITS, MT, CAP, AM><<<p.ctas_per_sm * sms, T, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -755,6 +765,8 @@ cudaError_t launch_copy(const StreamParams& p, int smem, cudaStream_t stream) {
   q.xbufs = p.xbufs;
   q.ctas_per_sm = p.ctas_per_sm;
   q.xbuf_bytes = p.xbuf_bytes;
+  q.max_polls = p.max_polls;
+  q.skip_first_copy = p.skip_first_copy;
   for (int i = 0; i < p.count; ++i) q.m[i] = p.m[i];
   return launch_cap<BITS, MT, CAP, AM>(q, smem, stream);
 }
@@ -793,6 +805,6 @@ cudaError_t launch_gemv_stream_argmax(const StreamParams& p, int bits, int smem,
   return bits == 4 ? launch_copy<4, 1, 1, true>(p, smem, stream) : launch_copy<2, 1, 1, true>(p, smem, stream);
 }
 
-int stream_grid(const StreamParams& p) { return p.ctas_per_sm * sm_count(); }
+int stream_grid(const StreamParams& p) { return p.ctas_per_sm * device_sm_count(); }
 
 }  // namespace wq

@@ -47,6 +47,8 @@ struct StreamParamsT {
   int xbufs;             // staged activation buffers per CTA (1 or 2)
   int ctas_per_sm;       // CTAs that fit on one SM with this set's shared memory
   int xbuf_bytes;        // bytes of one activation buffer
+  uint32_t max_polls;    // bound on the polls of one mbarrier wait
+  int skip_first_copy;   // failure-detection test: CTA 0's warp 0 never fills its first ring slot
   // fused argmax over the rows of a single matrix (null when not wanted): work space of
   // 16 + 8 * gridDim.x bytes whose first word is a CTA ticket counter (zero between calls),
   // followed by one (fp32 value, int32 row) partial per CTA; the result row goes to am_out

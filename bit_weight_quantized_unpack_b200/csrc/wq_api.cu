@@ -6,8 +6,10 @@
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "api_internal.cuh"
 #include "gemv_rows.cuh"
 #include "gemv_stream.cuh"
+#include "host_util.cuh"
 #include "wq.h"
 
 namespace {
@@ -31,19 +33,22 @@ namespace {
 // The kernels are built for sm_100a only: refuse any other device up front instead of
 // failing inside a launch. Cached per device ordinal.
 int check_device() {
-  static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+  static std::atomic<int> cached[wq::kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_status(e);
-  if (dev < 0 || dev >= 64) return WQ_ERR_UNSUPPORTED;
-  if (cached[dev] == 0) {
+  if (dev < 0 || dev >= wq::kMaxDevices) return WQ_ERR_UNSUPPORTED;
+  int c = cached[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
     int major = 0, minor = 0;
     e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     if (e != cudaSuccess) return cuda_status(e);
-    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    c = (major == 10 && minor == 0) ? 1 : 2;
+    cached[dev].store(c, std::memory_order_relaxed);
   }
-  return cached[dev] == 1 ? WQ_OK : WQ_ERR_UNSUPPORTED;
+  return c == 1 ? WQ_OK : WQ_ERR_UNSUPPORTED;
 }
 
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -85,6 +90,10 @@ int64_t plan_mat(wq::SetMat& m, int fmt, const void* codes, const uint16_t* scal
 // Streaming kernel for a set (int4 / int2) with M = 1 .. 4 rows of X: needs 16-byte aligned
 // codes, scales, zeros and activations, and activations short enough to stage in shared
 // memory.
+// Failure-detection test hook (wq_debug_arm_timeout): poll bound for the next streaming launch
+// on this thread, with one of its ring slots never filled; 0 = disarmed.
+thread_local uint32_t g_arm_polls = 0;
+
 int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStream_t stream, bool* done) {
   *done = false;
   if (count > wq::kStreamMaxMats || M > wq::kStreamMaxRows) return WQ_OK;
@@ -95,9 +104,16 @@ int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStrea
   const int smem = wq::stream_plan(sp, bits, count, sd, (int)M);
   if (smem == 0) return WQ_OK;
   *done = true;
+  if (g_arm_polls) {
+    sp.max_polls = g_arm_polls;
+    sp.skip_first_copy = 1;
+    g_arm_polls = 0;
+  }
   return cuda_status(wq::launch_gemv_stream(sp, bits, (int)M, smem, stream));
 }
 
+// Streaming tensor-core kernel for an int4 set with M = 1 .. 8 rows of X: needs 16-byte
+// aligned codes and activations, and K <= 32768 (activations staged in shared memory).
 // int3 set: one warp per output row (any M).
 int launch_int3(const wq_linear_desc* d, int count, cudaStream_t stream) {
   static thread_local wq::SetParams p;
@@ -157,6 +173,47 @@ int try_rows(int fmt, int count, const wq_linear_desc* d, cudaStream_t stream, b
 }
 
 }  // namespace
+
+namespace wq {
+
+namespace {
+// The plan of the last argmax_prepare on this thread (consumed by argmax_launch).
+thread_local StreamParams g_am_stream;
+thread_local int g_am_bits = 0;  // 0: no plan; 4 or 2: int4 / int2 on the streaming kernel
+thread_local int g_am_smem = 0;
+}  // namespace
+
+int argmax_prepare(const uint16_t* x, const void* codes, const uint16_t* scale, const uint16_t* zero, int fmt,
+                   int64_t N, int64_t K, uint16_t* y, int32_t* argmax, size_t* workspace_needed) {
+  g_am_bits = 0;
+  int st = check_shape(fmt, N, K);
+  if (st != WQ_OK) return st;
+  if (fmt == WQ_TERNARY || fmt == WQ_INT3 || !x || !argmax) return WQ_ERR_ARG;
+  if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scale, 16) || !aligned(zero, 16) ||
+      (y && !aligned(y, 2)) || !aligned(argmax, 4))
+    return WQ_ERR_ALIGN;
+  if (K > 32768) return WQ_ERR_SHAPE;
+  if ((st = check_device()) != WQ_OK) return st;
+  const int bits = fmt == WQ_INT4 ? 4 : 2;
+  const StreamDesc d = {codes, scale, zero, x, y, N, K};
+  g_am_smem = stream_plan(g_am_stream, bits, 1, &d, 1);
+  if (g_am_smem == 0) return WQ_ERR_SHAPE;
+  g_am_stream.am_out = reinterpret_cast<int*>(argmax);
+  *workspace_needed = 16 + 8 * (size_t)stream_grid(g_am_stream);
+  g_am_bits = bits;
+  return WQ_OK;
+}
+
+int argmax_launch(void* workspace, cudaStream_t stream) {
+  const int bits = g_am_bits;
+  g_am_bits = 0;
+  if (bits == 0) return WQ_ERR_ARG;
+  g_am_stream.am_ws = static_cast<unsigned int*>(workspace);
+  return note_cuda_error(launch_gemv_stream_argmax(g_am_stream, bits, g_am_smem, stream));
+}
+
+}  // namespace wq
 
 extern "C" {
 
@@ -334,33 +391,21 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
 
 size_t wq_argmax_workspace_bytes(void) {
   if (check_device() != WQ_OK) return 0;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return 0;
+  const int sms = wq::device_sm_count();
+  if (sms == 0) return 0;
   return 16 + 8 * (size_t)wq::kStreamMaxCtasPerSm * (size_t)sms;
 }
 
 int wq_gemv_argmax(const uint16_t* x, const void* codes, const uint16_t* scale, const uint16_t* zero, int fmt,
                    int64_t N, int64_t K, uint16_t* y, int32_t* argmax, void* workspace, size_t workspace_bytes,
                    void* stream) {
-  int st = check_shape(fmt, N, K);
+  if (!workspace) return WQ_ERR_ARG;
+  if (!aligned(workspace, 16)) return WQ_ERR_ALIGN;
+  size_t need = 0;
+  const int st = wq::argmax_prepare(x, codes, scale, zero, fmt, N, K, y, argmax, &need);
   if (st != WQ_OK) return st;
-  if (fmt == WQ_TERNARY || fmt == WQ_INT3 || !x || !argmax || !workspace) return WQ_ERR_ARG;
-  if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
-  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scale, 16) || !aligned(zero, 16) ||
-      !aligned(workspace, 16) || (y && !aligned(y, 2)) || !aligned(argmax, 4))
-    return WQ_ERR_ALIGN;
-  if (K > 32768) return WQ_ERR_SHAPE;
-  if ((st = check_device()) != WQ_OK) return st;
-  static thread_local wq::StreamParams sp;
-  const wq::StreamDesc d = {codes, scale, zero, x, y, N, K};
-  const int bits = fmt == WQ_INT4 ? 4 : 2;
-  const int smem = wq::stream_plan(sp, bits, 1, &d, 1);
-  if (smem == 0) return WQ_ERR_SHAPE;
-  if (workspace_bytes < 16 + 8 * (size_t)wq::stream_grid(sp)) return WQ_ERR_ARG;
-  sp.am_ws = static_cast<unsigned int*>(workspace);
-  sp.am_out = reinterpret_cast<int*>(argmax);
-  return cuda_status(wq::launch_gemv_stream_argmax(sp, bits, smem, (cudaStream_t)stream));
+  if (workspace_bytes < need) return WQ_ERR_ARG;
+  return wq::argmax_launch(workspace, (cudaStream_t)stream);
 }
 
 const char* wq_status_str(int status) {
@@ -377,6 +422,11 @@ const char* wq_status_str(int status) {
 }
 
 int wq_last_cuda_error(void) { return g_last_cuda_error; }
+
+int wq_debug_arm_timeout(unsigned int polls) {
+  g_arm_polls = polls;
+  return WQ_OK;
+}
 
 int wq_device_errors(unsigned int* flags, int clear, void* stream) {
   if (!flags) return WQ_ERR_ARG;

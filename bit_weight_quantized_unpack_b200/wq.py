@@ -45,6 +45,7 @@ _sig = {
     "wq_status_str": (ctypes.c_char_p, [_i]),
     "wq_last_cuda_error": (_i, []),
     "wq_device_errors": (_i, [ctypes.POINTER(ctypes.c_uint), _i, _p]),
+    "wq_debug_arm_timeout": (_i, [ctypes.c_uint]),
     "wq_argmax_workspace_bytes": (ctypes.c_size_t, []),
     "wq_gemv_argmax": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p, _p, ctypes.c_size_t, _p]),
     "wq_gemv_argmax_static": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p, _p]),
@@ -177,6 +178,12 @@ def wq_device_errors(clear: bool = True, stream=None) -> int:
 
 
 WQ_DEVERR_TIMEOUT = 1
+
+
+def wq_debug_arm_timeout(polls: int) -> None:
+    """Failure-detection test hook: the next streaming-kernel launch on this thread has one
+    unfilled ring slot and waits of at most `polls` polls (0 disarms)."""
+    _check(_lib.wq_debug_arm_timeout(int(polls)), "wq_debug_arm_timeout")
 
 
 # ---- allocation helpers (torch owns the memory) ------------------------------------

@@ -208,11 +208,24 @@ const char* wq_status_str(int status);
 int wq_last_cuda_error(void);
 
 /* Device-side error flags of this library on the current device, OR-ed over every kernel
- * since the last clear: bit 0 (WQ_DEVERR_TIMEOUT) = a bounded wait inside a tensor-core
- * kernel gave up (its outputs are then undefined; the kernel freed its resources and
- * returned instead of hanging). Synchronises `stream`; clears the flags if clear != 0. */
+ * since the last clear: bit 0 (WQ_DEVERR_TIMEOUT) = a bounded wait on an mbarrier inside a
+ * kernel (the streaming matrix-vector kernel, the tensor-core GEMM) gave up; that launch's
+ * outputs are undefined, and the kernel stopped computing, waited (bounded) for its copies
+ * still in flight, freed its tensor memory and returned instead of hanging. Kernels run
+ * after their call has returned, so a timeout cannot be a wq_status of that call; it is
+ * reported here. `flags` is a HOST pointer. Synchronises `stream`; clears the flags if
+ * clear != 0. */
 #define WQ_DEVERR_TIMEOUT 1u
 int wq_device_errors(unsigned int* flags, int clear, void* stream);
+
+/* Failure-detection test hook (no counterpart on the pages). Arms the next wq_gemv / wq_gemm /
+ * wq_linear_set call made on this host thread that launches the streaming matrix-vector
+ * kernel (int4 / int2 / ternary with M = 1 .. 4): in that launch, one ring slot of warp 0 of
+ * CTA 0 is never filled and every mbarrier wait gives up after `polls` polls. The wait on
+ * the unfilled slot therefore runs out, and the kernel takes its error path (WQ_DEVERR_TIMEOUT
+ * in wq_device_errors, outputs of that call undefined) without any GPU fault, trap or hang.
+ * The next call runs normally. polls = 0 disarms. Always returns WQ_OK. */
+int wq_debug_arm_timeout(unsigned int polls);
 
 #ifdef __cplusplus
 }
