@@ -12,8 +12,8 @@ float64. Where the pages leave a step open, the plainest reading is taken and ma
 READING in the function's docstring.
 
 Pins (tests/test_oracle_pins.py): the parameter and bytes/token tables of "The one fact
-that shapes everything", bits/weight of the format tables, the 243-code base-3 round
-trip, the +-1 XOR/popcount identity of "Measured hardware facts", closed-form quantiser
+that shapes everything", bits/weight of the format tables (int4 hier-g32 4.28 on the 0.5B
+set and 4.26 on the 7B set included), the 243-code base-3 round trip, the +-1 XOR/popcount identity of "Measured hardware facts", closed-form quantiser
 cases, an exhaustive check of the fp16 rounding routine, and exact rational products.
 Parity unpinned: nothing in the quality tables of "What the weights can actually survive"
 (they need trained checkpoints).
@@ -273,6 +273,85 @@ def dequant_ternary(packed, scale_bits, K: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
+# Hierarchical int4, group 32.  Whetstone README, "What the weights can actually survive":
+# group 32 with an fp16 scale and zero per group would cost 1.0 bits/weight of metadata,
+# so the format stores two 4-bit indices per group against one f16 pair per row (format
+# table of "The one fact that shapes everything": "int4 hier-g32", 4.28 bits/weight);
+# "Prior art": the same idea as GGUF Q4_K, sub-block scale and min indices against a
+# super-block f16 pair; "New in 0.6.0": the shared fp16 row scale could underflow to zero
+# and garble whole rows (seen only on the 7B model).
+# --------------------------------------------------------------------------------------
+HIER_GROUP = 32
+F16_TINY = 2.0 ** -24  # smallest positive binary16
+
+
+def _row_scale(num):
+    """fp16(num / 15) for the row pair, with the underflow guard: a positive numerator whose
+    quotient rounds to 0 gives the smallest positive binary16 instead, and a zero numerator
+    (nothing to scale) gives 1."""
+    d = f16_round(num / 15.0)
+    d = np.where((d == 0.0) & (num > 0.0), F16_TINY, d)
+    return np.where(num == 0.0, 1.0, d)
+
+
+def quantize_int4h(W):
+    """Hierarchical int4 quantisation: 4-bit codes in groups of 32 along K, each group's
+    scale and min given by two 4-bit indices into one fp16 pair (d, dm) per row.
+
+    READING (the pages give the geometry -- group 32, two 4-bit indices per group, an f16
+    pair per row -- and the Q4_K analogy, not a formula). Round to nearest throughout, per
+    row n, in float64:
+        per group g (32 consecutive k):  lo = min w, hi = max w
+            m_g = max(0, -lo)                the group's min offset (Q4_K style, never < 0)
+            s_g = (hi + m_g) / 15            the step that spans [-m_g, hi]
+        d  = fp16(max_g s_g / 15),  dm = fp16(max_g m_g / 15)      (with _row_scale's guard)
+        a_g = clamp(rint(s_g / d), 0, 15),   b_g = clamp(rint(m_g / dm), 0, 15)
+        S_g = d a_g,  Z_g = dm b_g           (exact: an fp16 value times a 4-bit integer)
+        q   = clamp(rint((w + Z_g) / S_g), 0, 15)   (q = 0 where S_g = 0)
+    and w_hat = S_g q - Z_g. rint is ties-to-even; w + Z_g and the quotients are float64
+    operations, rounded once each, in this order.
+    Returns codes uint32 [N, K/8] (the int4 layout: code k in word k/8, bits 4(k%8)),
+    pair uint16 [N, 2] (fp16 bits of d, dm) and idx uint8 [N, K/32] (a_g | b_g << 4).
+    """
+    W = np.asarray(W)
+    N, K = W.shape
+    assert K % GROUP == 0
+    G = K // HIER_GROUP
+    w = W.astype(np.float64).reshape(N, G, HIER_GROUP)
+    lo = w.min(axis=2)
+    hi = w.max(axis=2)
+    m = np.maximum(0.0, -lo)
+    s = (hi + m) / 15.0
+    d = _row_scale(s.max(axis=1))
+    dm = _row_scale(m.max(axis=1))
+    a = np.clip(np.rint(s / d[:, None]), 0.0, 15.0)
+    b = np.clip(np.rint(m / dm[:, None]), 0.0, 15.0)
+    S = d[:, None] * a
+    Z = dm[:, None] * b
+    safe = np.where(S > 0.0, S, 1.0)
+    q = np.clip(np.rint((w + Z[:, :, None]) / safe[:, :, None]), 0.0, 15.0)
+    q = np.where((S > 0.0)[:, :, None], q, 0.0).astype(np.uint32)
+    pair = np.stack([f16_to_bits(d), f16_to_bits(dm)], axis=1)
+    idx = (a.astype(np.uint32) | (b.astype(np.uint32) << 4)).astype(np.uint8)
+    return pack_int(q.reshape(N, K), 4), pair, idx
+
+
+def dequant_int4h(codes, pair_bits, idx, K: int) -> np.ndarray:
+    """w_hat[n, k] = d_n a_g q - dm_n b_g for k in group g (float64, exact)."""
+    q = unpack_int(codes, 4, K).astype(np.float64)
+    pr = f16_from_bits(np.asarray(pair_bits, dtype=np.uint16))
+    ix = np.asarray(idx, dtype=np.int64)
+    S = pr[:, 0:1] * (ix & 15).astype(np.float64)
+    Z = pr[:, 1:2] * (ix >> 4).astype(np.float64)
+    return q * np.repeat(S, HIER_GROUP, axis=1) - np.repeat(Z, HIER_GROUP, axis=1)
+
+
+def int4h_bytes(N: int, K: int) -> int:
+    """Stored bytes of an [N, K] int4h weight: codes + one index byte per 32 + fp16 pair per row."""
+    return N * K // 2 + N * K // HIER_GROUP + 4 * N
+
+
+# --------------------------------------------------------------------------------------
 # The product.  Whetstone README, "The one fact that shapes everything": at batch 1 every
 # weight is read once and used for one multiply-add; "Evaluation harness": float64
 # throughout.  y = x . w_hat^T, with the fp16 activations taken as exact float64 values.
@@ -292,9 +371,12 @@ def linear(x, w_hat):
 
 
 def gemv_packed(x, fmt: str, packed, scale_bits, zero_bits, K: int):
-    """Dequantise packed weights, then linear(); fmt in {'int4', 'int2', 'ternary'}."""
+    """Dequantise packed weights, then linear(); fmt in {'int4', 'int3', 'int2', 'ternary',
+    'int4h'} (for 'int4h' scale_bits is the row pair and zero_bits the index bytes)."""
     if fmt == "ternary":
         w_hat = dequant_ternary(packed, scale_bits, K)
+    elif fmt == "int4h":
+        w_hat = dequant_int4h(packed, scale_bits, zero_bits, K)
     else:
         w_hat = dequant_int(packed, scale_bits, zero_bits, INT_BITS[fmt], K)
     return linear(x, w_hat)
@@ -305,6 +387,8 @@ def quantize(W, fmt: str):
     if fmt == "ternary":
         p, s = quantize_ternary(W)
         return p, s, None
+    if fmt == "int4h":
+        return quantize_int4h(W)
     return quantize_int(W, INT_BITS[fmt])
 
 
@@ -383,8 +467,11 @@ def tok_s_ceiling(bandwidth_bytes_per_s: float, bytes_per_token_: float) -> floa
     return bandwidth_bytes_per_s / bytes_per_token_
 
 
-def stored_bits_per_weight(fmt: str) -> float:
-    """Bits per weight of this layout as stored: codes + fp16 metadata per 128 weights."""
+def stored_bits_per_weight(fmt: str, K: int | None = None) -> float:
+    """Bits per weight of this layout as stored: codes + fp16 metadata per 128 weights
+    (int4h: codes + one index byte per 32 weights + one fp16 pair per row of K)."""
+    if fmt == "int4h":
+        return 4 + 8 / HIER_GROUP + 32 / K
     if fmt == "ternary":
         return (TERNARY_GROUP_BYTES * 8 + 16) / GROUP
     return INT_BITS[fmt] + 32 / GROUP
