@@ -155,7 +155,7 @@ def build_set(widx, copies, fmt="int4"):
             seed = synth.sub_seed(wl["seed"] + 7919 * cidx, i, 0)
             W = synth.weights(m.N, m.K, wl["sigma"], seed, device="cuda")
             c, s, z = wq.alloc_packed(m.N, m.K, fmt)
-            wq.wq_quantize(W, m.N, m.K, fmt, 128, c, s, z)
+            wq.wq_quantize(W, m.N, m.K, fmt, 32 if fmt == "int4h" else 128, c, s, z)
             del W
             x = x_all[ko:ko + m.K]
             x.copy_(synth.activations(1, m.K, synth.sub_seed(wl["seed"], i, 1), device="cuda")[0])
@@ -202,7 +202,7 @@ def bench_rows(args, pk):
     N, K = 151936, 896
     wl = workloads.WORKLOADS[2]
     # lm_head alone, each format; 4+ rotating copies so the working set exceeds L2
-    for fmt in ("int4", "int3", "int2", "ternary"):
+    for fmt in ("int4", "int4h", "int3", "int2", "ternary"):
         copies = []
         for cidx in range(6 if fmt != "int4" else 4):
             W = synth.weights_with_outliers(N, K, wl["sigma"], synth.sub_seed(wl["seed"] + cidx, 0, 0),
@@ -219,12 +219,12 @@ def bench_rows(args, pk):
                 torch.cuda.synchronize()
                 ms = ev0.elapsed_time(ev1) / 5
                 rows["quantize_int4_lm_head"] = {"ms": ms, "W_GBps": N * K * 4 / ms / 1e6}
-            wq.wq_quantize(W, N, K, fmt, 128, c, s, z)
+            wq.wq_quantize(W, N, K, fmt, 32 if fmt == "int4h" else 128, c, s, z)
             del W
             copies.append((c, s, z))
         x = synth.activations(1, K, 99, device="cuda")[0]
         y = torch.empty(N, dtype=torch.float16, device="cuda")
-        nb = wq.wq_codes_bytes(fmt, N, K) + 2 * wq.wq_meta_count(N, K) * (1 if fmt == "ternary" else 2)
+        nb = wq.wq_codes_bytes(fmt, N, K) + wq.wq_scale_bytes(fmt, N, K) + wq.wq_zero_bytes(fmt, N, K)
 
         def step(i, copies=copies, fmt=fmt):
             c, s, z = copies[i % len(copies)]
@@ -262,9 +262,30 @@ def bench_rows(args, pk):
             del w16
         del copies
         torch.cuda.empty_cache()
+    rows.update(bench_int4h_set(args, pk))
     rows.update(bench_batch_sweep(args, pk))
     rows.update(bench_7b_set(args, pk))
     return rows
+
+
+def bench_int4h_set(args, pk):
+    """The 0.5B decode set in hierarchical int4 (group-32 indices against a per-row fp16 pair,
+    4.28 bits/weight): one wq_linear_set per token, 2 rotating copies (each larger than L2)."""
+    from bit_weight_quantized_unpack_b200 import wq
+    sets, weights, _, _ = build_set(1, copies=2, fmt="int4h")
+    nbytes = sum(wq.wq_codes_bytes("int4h", m.N, m.K) + wq.wq_scale_bytes("int4h", m.N, m.K) +
+                 wq.wq_zero_bytes("int4h", m.N, m.K) for m in workloads.workload_mats(1))
+
+    def step(i):
+        s = sets[i % len(sets)]
+        wq.wq_linear_set(s["desc"], s["count"], "int4h")
+    ms = time_steps(step, 200 if not args.quick else 20, 10, 1)
+    out = {"gemv_set_qwen05b_int4h": {"ms": ms, "GBps": nbytes / ms / 1e6,
+                                      "frac_hbm": nbytes / ms / 1e6 / pk["hbm_gbs"],
+                                      "bytes_per_token": nbytes, "implied_tok_s": 1e3 / ms}}
+    del sets
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_7b_set(args, pk):

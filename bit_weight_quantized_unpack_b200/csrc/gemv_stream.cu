@@ -1,4 +1,5 @@
-// Matrix-vector product against packed int4 / int2 weights, streamed as contiguous bytes.
+// Matrix-vector product against packed int4 / int2 / ternary / hierarchical-int4 weights,
+// streamed as contiguous bytes.
 //
 // Whetstone README, "The one fact that shapes everything": at batch 1 every weight is read
 // once for one multiply-add, so the product runs at the speed the packed codes stream from
@@ -26,6 +27,12 @@
 // holds the part of a row that continues into the next step, and the lane holding a row's
 // last group writes y.
 //
+// Hierarchical int4 (Whetstone README, "What the weights can actually survive": groups of 32
+// with two 4-bit indices against an f16 pair per row) uses the int4 cells unchanged: a cell
+// of 128 weights is four groups of 32, one 16-byte chunk each, and its four index bytes form
+// the per-cell metadata word; no zero point is subtracted (w_hat = d a q - dm b), the group
+// sums of x are staged beside the activations, and the lane reads its row's (d, dm) itself.
+//
 // The activation vector of the matrix being processed is staged once per CTA; two buffers
 // let the next matrix's vector load while the current one is in use.
 #include <climits>
@@ -44,27 +51,33 @@ namespace {
 constexpr int W = kStreamWarps;
 constexpr int T = 32 * W;
 constexpr int TERN = 1;  // format tag of ternary (5 trits per byte, 26 bytes per group)
+constexpr int HIER = kStreamHier;  // hierarchical int4 (group-32 indices, per-row fp16 pair)
 
 // Chunk permutation of group g (XOR mask on the chunk index), shared by the codes reads and
 // the staged activation layout.
 template <int BITS>
 __host__ __device__ __forceinline__ int xrot(int g) {
-  return BITS == 4 ? (g >> 1) & 3 : BITS == 2 ? (g >> 2) & 1 : 0;
+  return (BITS == 4 || BITS == HIER) ? (g >> 1) & 3 : BITS == 2 ? (g >> 2) & 1 : 0;
 }
 
-// Per format (BITS = 4, 2, or TERN): bytes of codes per cell (one group), ring slot layout
-// (codes, then scales, then zeros for the integer formats), staged activation units per group.
+// Per format (BITS = 4, 2, TERN or HIER): bytes of codes per cell (128 weights of a row), ring
+// slot layout (codes, then the per-cell metadata: scales and zeros of the g128 integer
+// formats, scales of ternary, the four index bytes of HIER), staged activation units per group.
 template <int BITS>
 struct Fmt {
   static constexpr bool TRN = BITS == TERN;
-  static constexpr int CB = TRN ? 26 : 128 * BITS / 8;  // codes bytes per cell: 64 / 32 / 26
+  static constexpr bool HR = BITS == HIER;
+  static constexpr int CB = TRN ? 26 : HR ? 64 : 128 * BITS / 8;  // codes bytes per cell: 64 / 32 / 26
   static constexpr int CH = TRN ? 1 : CB / 16;          // 16-byte chunks per cell: 4 / 2
   static constexpr int UPC = 16 / CH;                   // activation units per chunk: 4 / 8
   static constexpr int SPS = TRN ? 4 : kStreamSlotCodes / (32 * CB);  // steps of 32 cells per slot
   static constexpr int SC = 32 * SPS * CB;              // codes bytes per slot: 4096 / 4096 / 3328
   static constexpr int GPSL = 32 * SPS;                 // groups per ring slot: 64 / 128 / 128
-  static constexpr int META = 2 * GPSL;                 // bytes of scales (and of zeros) per slot
-  static constexpr int SLOT = SC + (TRN ? 1 : 2) * META;
+  static constexpr int MB0 = HR ? 4 : 2;                // bytes per cell of metadata array 0 (scale / index)
+  static constexpr int MB1 = (TRN || HR) ? 0 : 2;       // bytes per cell of metadata array 1 (zero)
+  static constexpr int META0 = MB0 * GPSL;              // bytes of metadata array 0 per slot
+  static constexpr int META1 = MB1 * GPSL;
+  static constexpr int SLOT = SC + META0 + META1;
   static constexpr int XU = TRN ? 27 : 17;              // staged activation units per group
   static constexpr int LUT = TRN ? 256 * 4 : 0;         // byte -> five base-3 digits (shared memory)
 };
@@ -84,18 +97,19 @@ __device__ __forceinline__ uint16_t lds16(uint32_t a) {
 // at shared-memory address xa + m * xs), accumulated in binary32 with the factor 2^-24
 // described above. Each pair of codes is dequantised once for all MT rows.
 // int4: 32 codes; z1 / z16 hold z and 16 z as binary16 bit patterns in both lanes; the a
-// accumulators take codes at bits 0-3 of a byte, the b ones (16x) bits 4-7.
-template <int MT>
+// accumulators take codes at bits 0-3 of a byte, the b ones (16x) bits 4-7. SUBZ = false
+// (no zero point to subtract, the hierarchical format) leaves the masked codes as they are.
+template <int MT, bool SUBZ = true>
 __device__ __forceinline__ void chunk_int4(const uint4 c, uint32_t xa, uint32_t xs, uint32_t z1, uint32_t z16,
                                            float (&a)[MT][2], float (&b)[MT][2]) {
   const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t v = cw[i], v8 = v >> 8;
-    const uint32_t d0 = hsub2_u32(v & 0x000F000Fu, z1);    // q0, q4
-    const uint32_t d1 = hsub2_u32(v & 0x00F000F0u, z16);   // 16 q1, 16 q5
-    const uint32_t d2 = hsub2_u32(v8 & 0x000F000Fu, z1);   // q2, q6
-    const uint32_t d3 = hsub2_u32(v8 & 0x00F000F0u, z16);  // 16 q3, 16 q7
+    const uint32_t d0 = SUBZ ? hsub2_u32(v & 0x000F000Fu, z1) : v & 0x000F000Fu;     // q0, q4
+    const uint32_t d1 = SUBZ ? hsub2_u32(v & 0x00F000F0u, z16) : v & 0x00F000F0u;   // 16 q1, 16 q5
+    const uint32_t d2 = SUBZ ? hsub2_u32(v8 & 0x000F000Fu, z1) : v8 & 0x000F000Fu;   // q2, q6
+    const uint32_t d3 = SUBZ ? hsub2_u32(v8 & 0x00F000F0u, z16) : v8 & 0x00F000F0u;  // 16 q3, 16 q7
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       const uint4 xw = lds128(xa + m * xs + 16 * i);  // (x0, x1) (x2, x3) (x4, x5) (x6, x7)
@@ -213,6 +227,44 @@ __device__ __forceinline__ void cell_dot_ternary(uint32_t cell, uint32_t xg, uin
   for (int m = 0; m < MT; ++m) out[m] = a[m][0] + a[m][1];
 }
 
+// Hierarchical int4 (one cell = 128 weights of a row = four groups of 32, one 16-byte chunk
+// each): P[m] = 2^-24 sum_j a_j sum_{k in group j} x_mk q_k and Q[m] = sum_j b_j sum_{k in
+// group j} x_mk, so that the cell's share of y is d 2^24 P - dm Q (w_hat = d a_j q - dm b_j).
+// ib: the cell's four index bytes (a_j | b_j << 4, group j in byte j); rot: the cell's chunk
+// permutation (chunk c of the read order is group c ^ rot); the group sums of x are staged as
+// four binary32 values (group order) in the spare unit 16 of the cell's activation units.
+// The masked codes are the binary16 subnormals q 2^-24 (16 q 2^-24 for bits 4-7), so each
+// product with x is exact in binary32, as for int4.
+__device__ __forceinline__ float small_int_f32(uint32_t v) {  // exact float of 0 <= v < 2^23
+  return __uint_as_float(0x4B000000u | v) - 8388608.0f;
+}
+
+template <int MT>
+__device__ __forceinline__ void cell_dot_hier(uint32_t cell, uint32_t xg, uint32_t xs, const int (&oc)[4],
+                                              const int (&ox)[4], int rot, uint32_t ib, float (&P)[MT],
+                                              float (&Q)[MT]) {
+#pragma unroll
+  for (int m = 0; m < MT; ++m) P[m] = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float aj = small_int_f32((ib >> (8 * (c ^ rot))) & 15u);
+    float a[MT][2], b[MT][2];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) a[m][0] = a[m][1] = b[m][0] = b[m][1] = 0.f;
+    chunk_int4<MT, false>(lds128(cell + oc[c]), xg + ox[c], xs, 0u, 0u, a, b);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) P[m] = fmaf(aj, fmaf(b[m][0] + b[m][1], 0.0625f, a[m][0] + a[m][1]), P[m]);
+  }
+  const float b0 = small_int_f32((ib >> 4) & 15u), b1 = small_int_f32((ib >> 12) & 15u);
+  const float b2 = small_int_f32((ib >> 20) & 15u), b3 = small_int_f32(ib >> 28);
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const uint4 sx = lds128(xg + m * xs + 16 * 16);
+    Q[m] = fmaf(b3, __uint_as_float(sx.w),
+                fmaf(b2, __uint_as_float(sx.z), fmaf(b1, __uint_as_float(sx.y), b0 * __uint_as_float(sx.x))));
+  }
+}
+
 // Wait for an mbarrier phase, giving up after max_polls polls (false).
 __device__ __forceinline__ bool mbar_wait_n(uint32_t bar, uint32_t parity, uint32_t max_polls) {
   for (uint32_t i = 0; i < max_polls; ++i)
@@ -248,10 +300,11 @@ __device__ __forceinline__ void cta_units(const StreamMat& M, int64_t lo, int64_
 }
 
 // One warp's share of a matrix: whole units [wb0, wb1) of the CTA's range, as rows.
+// m0 / m1: the segment's per-cell metadata arrays (scales and zeros; HIER: index bytes, none).
 struct Seg {
   const uint8_t* codes;
-  const uint16_t* s;
-  const uint16_t* z;
+  const uint8_t* m0;
+  const uint8_t* m1;
   int rows;
   int row0;
   int bytes;   // codes bytes
@@ -270,8 +323,10 @@ __device__ __forceinline__ Seg warp_seg(const StreamMat& M, int b0, int b1, int 
   s.rows = r1 > r0 ? (int)(r1 - r0) : 0;
   s.row0 = (int)r0;
   s.codes = reinterpret_cast<const uint8_t*>(M.codes) + r0 * rb;
-  s.s = M.scale + r0 * G;
-  s.z = M.zero + r0 * G;
+  // HIER: the index bytes (passed as `zero`) are the per-cell metadata; the row pairs (passed
+  // as `scale`) are read by the consumer lanes
+  s.m0 = reinterpret_cast<const uint8_t*>(Fmt<BITS>::HR ? M.zero : M.scale) + r0 * G * Fmt<BITS>::MB0;
+  s.m1 = reinterpret_cast<const uint8_t*>(M.zero) + r0 * G * Fmt<BITS>::MB1;
   s.bytes = (int)(s.rows * rb);
   s.groups = s.rows * G;
   return s;
@@ -281,8 +336,8 @@ __device__ __forceinline__ Seg warp_seg(const StreamMat& M, int b0, int b1, int 
 // segment being issued.
 struct Prod {
   const uint8_t* c;
-  const uint16_t* s;
-  const uint16_t* z;
+  const uint8_t* m0;
+  const uint8_t* m1;
   int cleft;  // codes bytes not yet issued
   int gleft;  // groups not yet issued
   int pm;     // matrix of the segment
@@ -303,20 +358,25 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
   const int nsteps = (ncells + 31) / 32;
   const int nslots = (nsteps + F::SPS - 1) / F::SPS;
   uint16_t* y = M.y + seg.row0;
-  // the matrix's last partial 16-byte unit of scales / zeros, if this segment ends there:
-  // loaded now, stored into its ring slot before that slot is read
-  const int rem = ncells & 7;
+  // the matrix's last partial 16-byte unit of each metadata array, if this segment ends there:
+  // loaded now, stored into its ring slot before that slot is read (a unit holds 16 / MB0
+  // cells of array 0: 8, or 4 for HIER; array 1, where present, has MB1 = MB0 = 2)
+  const int rem = ncells & (16 / F::MB0 - 1);
   // ternary rows are 26 K / 128 bytes: a segment at the end of a matrix may end inside a
   // 16-byte unit; those last bytes are loaded here too
   const int crem = F::TRN ? (int)(seg.bytes & 15) : 0;
   uint32_t cr = 0;
   if (F::TRN && crem && lane >= 16 && lane < 16 + crem)
     cr = __ldg(seg.codes + (seg.bytes & ~(int64_t)15) + (lane - 16));
-  uint16_t rs = 0, rz = 0;
+  uint32_t rs = 0;
+  uint16_t rz = 0;
   if (rem) {
     const int gb = ncells - rem;
-    if (lane < rem) rs = ld_u16(seg.s + gb + lane);
-    if (!F::TRN && lane >= 8 && lane < 8 + rem) rz = ld_u16(seg.z + gb + lane - 8);
+    if (lane < rem) {
+      if constexpr (F::MB0 == 4) rs = __ldg(reinterpret_cast<const uint32_t*>(seg.m0) + gb + lane);
+      else rs = ld_u16(reinterpret_cast<const uint16_t*>(seg.m0) + gb + lane);
+    }
+    if (F::MB1 && lane >= 8 && lane < 8 + rem) rz = ld_u16(reinterpret_cast<const uint16_t*>(seg.m1) + gb + lane - 8);
   }
   // group gp of row `row` of the segment: this lane's cell
   const uint32_t gmul = ((1u << 20) + G - 1) / G;  // floor(n / G) = (n * gmul) >> 20 for n < G + 32, G < 32
@@ -344,13 +404,18 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
     }
     if (rem && k == nslots - 1) {
       const int gl = ncells - rem - k * F::GPSL;
-      if (lane < rem) asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + F::SC + 2 * (gl + lane)), "h"(rs));
-      if (!F::TRN && lane >= 8 && lane < 8 + rem)
-        asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + F::SC + F::META + 2 * (gl + lane - 8)), "h"(rz));
+      if (lane < rem) {
+        if constexpr (F::MB0 == 4)
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(slot + F::SC + 4 * (gl + lane)), "r"(rs));
+        else
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + F::SC + 2 * (gl + lane)), "h"((uint16_t)rs));
+      }
+      if (F::MB1 && lane >= 8 && lane < 8 + rem)
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(slot + F::SC + F::META0 + 2 * (gl + lane - 8)), "h"(rz));
       tc::fence_proxy_async_smem();  // the slot is refilled by bulk copies later
       __syncwarp();
     }
-    const uint32_t cell0 = slot + lane * F::CB, meta0 = slot + F::SC + 2 * lane;
+    const uint32_t cell0 = slot + lane * F::CB, meta0 = slot + F::SC + F::MB0 * lane;
 #pragma unroll
     for (int ss = 0; ss < F::SPS; ++ss) {
       const int st = k * F::SPS + ss;
@@ -359,7 +424,27 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
       float v[MT];
 #pragma unroll
       for (int m = 0; m < MT; ++m) v[m] = 0.f;
-      if (valid && !dead) {
+      if constexpr (F::HR) {
+        if (valid && !dead) {
+          // the row's pair (d, dm): read here, used after the cell's products
+          const uint32_t pr = __ldg(reinterpret_cast<const uint32_t*>(M.scale) + seg.row0 + row);
+          uint32_t ib;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ib) : "r"(meta0 + 32 * F::MB0 * ss));
+          const int rot = xrot<BITS>(gp);
+          int oc[4], ox[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            oc[c] = 16 * (c ^ rot);
+            ox[c] = 16 * F::UPC * c;
+          }
+          float Pv[MT], Qv[MT];
+          cell_dot_hier<MT>(cell0 + 32 * F::CB * ss, xb + 16 * F::XU * gp, xs, oc, ox, rot, ib, Pv, Qv);
+          const float d24 = __half2float(__ushort_as_half(lo16(pr))) * 16777216.f;  // 2^24 back, exactly
+          const float dm = __half2float(__ushort_as_half(hi16(pr)));
+#pragma unroll
+          for (int m = 0; m < MT; ++m) v[m] = fmaf(Pv[m], d24, -(Qv[m] * dm));
+        }
+      } else if (valid && !dead) {
         const uint16_t sb = lds16(meta0 + 64 * ss);
         if constexpr (F::TRN) {
           cell_dot_ternary<MT>(cell0 + 32 * F::CB * ss, xb + 16 * F::XU * gp, xs, lut, v);
@@ -367,7 +452,7 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
 #pragma unroll
           for (int m = 0; m < MT; ++m) v[m] *= sf;
         } else {
-        const uint16_t zb = lds16(meta0 + 64 * ss + F::META);
+        const uint16_t zb = lds16(meta0 + 64 * ss + F::META0);
         // chunks in an order permuted by the group index, so that the lanes of one
         // shared-memory phase (consecutive cells) hit different bank groups; the staged
         // activations of each group are stored in that same order (see stage_x), so the
@@ -502,8 +587,8 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
       cta_units(M, lo, hi, b0, b1);
       const Seg sg = warp_seg<BITS>(M, b0, b1, w);
       pd.c = sg.codes;
-      pd.s = sg.s;
-      pd.z = sg.z;
+      pd.m0 = sg.m0;
+      pd.m1 = sg.m1;
       pd.cleft = sg.bytes;
       pd.gleft = sg.groups;
     }
@@ -513,21 +598,22 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
       cb = pd.cleft;
       gc = pd.gleft;
     }
-    // whole 16-byte units of scales / zeros (and, for ternary, of codes); the rest, at the
-    // end of a matrix, is loaded by the consumer lanes
-    const uint32_t mb = 2u * (uint32_t)(gc & ~7);
+    // whole 16-byte units of the metadata arrays (and, for ternary, of codes); the rest, at
+    // the end of a matrix, is loaded by the consumer lanes
+    const uint32_t units = (uint32_t)(gc & ~(16 / F::MB0 - 1));  // cells in whole units
+    const uint32_t mb0 = F::MB0 * units, mb1 = F::MB1 * units;
     const uint32_t cbb = (uint32_t)cb & ~15u;
     if (!(skip_first && issued == 0)) {
-      if (lane == 0) tc::mbar_arrive_expect_tx(bar, cbb + (F::TRN ? 1 : 2) * mb);
-      if (lane == 0 || (lane < (F::TRN ? 2 : 3) && mb)) {
-        const void* src = lane == 0 ? (const void*)pd.c : lane == 1 ? (const void*)pd.s : (const void*)pd.z;
-        const uint32_t d = lane == 0 ? dst : dst + F::SC + (lane - 1) * F::META;
-        bulk_g2s(d, src, lane == 0 ? cbb : mb, bar);
+      if (lane == 0) tc::mbar_arrive_expect_tx(bar, cbb + mb0 + mb1);
+      if (lane == 0 || (lane == 1 && mb0) || (F::MB1 && lane == 2 && mb1)) {
+        const void* src = lane == 0 ? (const void*)pd.c : lane == 1 ? (const void*)pd.m0 : (const void*)pd.m1;
+        const uint32_t d = lane == 0 ? dst : lane == 1 ? dst + F::SC : dst + F::SC + F::META0;
+        bulk_g2s(d, src, lane == 0 ? cbb : lane == 1 ? mb0 : mb1, bar);
       }
     }
     pd.c += cb;
-    pd.s += gc;
-    pd.z += gc;
+    pd.m0 += F::MB0 * gc;
+    pd.m1 += F::MB1 * gc;
     pd.cleft -= cb;
     pd.gleft -= gc;
     ++issued;
@@ -582,6 +668,27 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
                    : "memory");
     }
     cp_async_commit();
+    if constexpr (F::HR) {
+      // the sums of x over each group of 32, as binary32, in the spare unit 16 of the
+      // group's 17 (four per 128-weight cell, in group order)
+      const int ng = M.K / 32;
+      for (int t = threadIdx.x; t < MT * ng; t += T) {
+        const int m = t / ng, j = t - m * ng;
+        const uint4* src = reinterpret_cast<const uint4*>(M.x + (size_t)m * M.K + 32 * j);
+        float sum = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 q = __ldg(src + u);
+          const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            sum += __half2float(__ushort_as_half(lo16(qw[e]))) + __half2float(__ushort_as_half(hi16(qw[e])));
+        }
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(xb + 16 * (m * rowu + F::XU * (j >> 2) + 16) + 4 * (j & 3)),
+                     "f"(sum)
+                     : "memory");
+      }
+    }
   };
 
   float am_v = -INFINITY;  // fused argmax: this lane's best fp16 value and its row
@@ -695,14 +802,16 @@ int plan_t(StreamParams& p, int count, const StreamDesc* d, int mt) {
   int64_t cost = 0;
   int max_k = 0;
   for (int i = 0; i < count; ++i) {
-    if ((((uintptr_t)d[i].codes | (uintptr_t)d[i].scale | (uintptr_t)d[i].zero | (uintptr_t)d[i].x) & 15) != 0)
-      return 0;
+    // bulk-copied arrays 16-byte aligned; HIER row pairs are read as 4-byte words
+    const uintptr_t bulk = (uintptr_t)d[i].codes | (uintptr_t)d[i].zero | (uintptr_t)d[i].x |
+                           (F::HR ? 0 : (uintptr_t)d[i].scale);
+    if ((bulk & 15) != 0 || (F::HR && ((uintptr_t)d[i].scale & 3) != 0)) return 0;
     const int K = (int)d[i].K, N = (int)d[i].N;
     const int G = K / kGroup;
-    // rows per unit: segments start at multiples of RA rows, so that their scales and zeros
-    // start on a 16-byte boundary (8 groups)
-    const int RA = 8 / gcd_int(G, 8);
-    const int64_t row_cost = (int64_t)G * F::CB + (F::TRN ? 2 : 4) * G;
+    // rows per unit: segments start at multiples of RA rows, so that their metadata starts
+    // on a 16-byte boundary (a unit of 16 / MB0 cells)
+    const int RA = (16 / F::MB0) / gcd_int(G, 16 / F::MB0);
+    const int64_t row_cost = (int64_t)G * (F::CB + F::MB0 + F::MB1) + (F::HR ? 4 : 0);
     StreamMat& m = p.m[i];
     m.codes = d[i].codes;
     m.scale = d[i].scale;
@@ -793,16 +902,29 @@ cudaError_t launch_b(const StreamParams& p, int mt, int smem, cudaStream_t strea
 
 int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int mt) {
   if (count < 1 || count > kStreamMaxMats || mt < 1 || mt > kStreamMaxRows) return 0;
-  return bits == 4 ? plan_t<4>(p, count, d, mt) : bits == 2 ? plan_t<2>(p, count, d, mt) : plan_t<TERN>(p, count, d, mt);
+  switch (bits) {
+    case 4: return plan_t<4>(p, count, d, mt);
+    case 2: return plan_t<2>(p, count, d, mt);
+    case HIER: return plan_t<HIER>(p, count, d, mt);
+    default: return plan_t<TERN>(p, count, d, mt);
+  }
 }
 
 cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem, cudaStream_t stream) {
-  return bits == 4 ? launch_b<4>(p, mt, smem, stream)
-                   : bits == 2 ? launch_b<2>(p, mt, smem, stream) : launch_b<TERN>(p, mt, smem, stream);
+  switch (bits) {
+    case 4: return launch_b<4>(p, mt, smem, stream);
+    case 2: return launch_b<2>(p, mt, smem, stream);
+    case HIER: return launch_b<HIER>(p, mt, smem, stream);
+    default: return launch_b<TERN>(p, mt, smem, stream);
+  }
 }
 
 cudaError_t launch_gemv_stream_argmax(const StreamParams& p, int bits, int smem, cudaStream_t stream) {
-  return bits == 4 ? launch_copy<4, 1, 1, true>(p, smem, stream) : launch_copy<2, 1, 1, true>(p, smem, stream);
+  switch (bits) {
+    case 4: return launch_copy<4, 1, 1, true>(p, smem, stream);
+    case HIER: return launch_copy<HIER, 1, 1, true>(p, smem, stream);
+    default: return launch_copy<2, 1, 1, true>(p, smem, stream);
+  }
 }
 
 int stream_grid(const StreamParams& p) { return p.ctas_per_sm * device_sm_count(); }

@@ -67,7 +67,12 @@ struct StreamDesc {
   int64_t N, K;
 };
 
-// Fills p for a set of `count` matrices of one format (bits 4, 2, or 1 for ternary), each multiplied by mt
+// Format tags of the streaming kernel: bits 4 or 2 (g128 integer codes), 1 (ternary), 5
+// (hierarchical int4: codes as int4, `scale` the fp16 row pairs [N, 2], `zero` the index bytes
+// [N, K/32]).
+constexpr int kStreamHier = 5;
+
+// Fills p for a set of `count` matrices of one format (a tag above), each multiplied by mt
 // rows of X (X [mt, K] and Y [mt, N] row-major), and returns the bytes of dynamic shared
 // memory a CTA needs, or 0 if this kernel cannot serve the set (pointers not 16-byte
 // aligned, or activations too long to stage).

@@ -1,4 +1,5 @@
-// Group-128 quantisers (int4 / int3 / int2 asymmetric round-to-nearest, ternary absmean).
+// Quantisers: group-128 int4 / int3 / int2 asymmetric round-to-nearest, ternary absmean, and
+// hierarchical int4 with group-32 indices against a per-row fp16 pair.
 //
 // Whetstone README, "What the weights can actually survive": round-to-nearest with group
 // 128 and one fp16 scale plus one fp16 zero per group (format table rows "int4 g128",
@@ -133,8 +134,97 @@ __global__ void __launch_bounds__(256) quantize_ternary_kernel(const float* __re
   if (lane == 0) scale[task] = s_bits;
 }
 
+// Hierarchical int4, group 32 (Whetstone README, "What the weights can actually survive":
+// two 4-bit indices per group of 32 against one fp16 pair per row; "New in 0.6.0": the row
+// scale must not underflow to zero). The definition is per row (the pair depends on every
+// group of the row), so one warp takes one row in two passes: the row maxima of s_g and m_g,
+// then the indices and codes. Each pass reads 128 weights (four groups) per iteration;
+// lanes 8j .. 8j+7 hold group j of the iteration, four weights each.
+
+// rs(v) of the int4h definition: fp16(v / 15), 1 for v = 0, the smallest positive binary16
+// where a positive v rounds to zero.
+__device__ __forceinline__ uint16_t row_scale_bits(double v) {
+  if (v == 0.0) return 0x3C00;
+  const uint16_t b = f64_to_f16_bits(v / 15.0);
+  return b == 0 ? (uint16_t)0x0001 : b;
+}
+
+// lo and hi of the 32 weights held by a lane's group of eight lanes (four each)
+__device__ __forceinline__ void group32_minmax(const float4 v, float& lo, float& hi) {
+  lo = fminf(fminf(v.x, v.y), fminf(v.z, v.w));
+  hi = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+}
+
+__global__ void __launch_bounds__(256) quantize_int4h_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+                                                             uint32_t* __restrict__ codes,
+                                                             uint16_t* __restrict__ pair,
+                                                             uint8_t* __restrict__ idx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (n >= N) return;  // warp-uniform
+  const float* row = W + n * K;
+  const int iters = (int)(K / 128);
+
+  // pass 1: max_g s_g and max_g m_g (maxima are exact in any order)
+  double smax = 0.0, mmax = 0.0;
+  for (int it = 0; it < iters; ++it) {
+    const float4 v = *reinterpret_cast<const float4*>(row + 128 * it + 4 * lane);
+    float lo, hi;
+    group32_minmax(v, lo, hi);
+    const double m = fmax(0.0, -(double)lo);
+    const double sg = ((double)hi + m) / 15.0;
+    smax = fmax(smax, sg);
+    mmax = fmax(mmax, m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    smax = fmax(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+    mmax = fmax(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  }
+  const uint16_t d_bits = row_scale_bits(smax), dm_bits = row_scale_bits(mmax);
+  const double d = f16_bits_to_f64(d_bits), dm = f16_bits_to_f64(dm_bits);
+
+  // pass 2: indices and codes
+  for (int it = 0; it < iters; ++it) {
+    const float4 v = *reinterpret_cast<const float4*>(row + 128 * it + 4 * lane);
+    float lo, hi;
+    group32_minmax(v, lo, hi);
+    const double m = fmax(0.0, -(double)lo);
+    const double sg = ((double)hi + m) / 15.0;
+    const double a = fmin(fmax(rint(sg / d), 0.0), 15.0);
+    const double b = fmin(fmax(rint(m / dm), 0.0), 15.0);
+    const double S = d * a, Z = dm * b;  // exact: a binary16 value times a 4-bit integer
+    const float wv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const double q = S > 0.0 ? fmin(fmax(rint(((double)wv[i] + Z) / S), 0.0), 15.0) : 0.0;
+      packed |= (uint32_t)q << (4 * i);
+    }
+    // lanes 2j and 2j+1 hold codes 8j..8j+3 and 8j+4..8j+7 of the iteration's word j
+    packed <<= 16 * (lane & 1);
+    packed |= __shfl_xor_sync(0xffffffffu, packed, 1);
+    if ((lane & 1) == 0) codes[n * (K / 8) + 16 * it + (lane >> 1)] = packed;
+    if ((lane & 7) == 0) idx[n * (K / 32) + 4 * it + (lane >> 3)] = (uint8_t)((uint32_t)a | (uint32_t)b << 4);
+  }
+  if (lane == 0) {
+    pair[2 * n] = d_bits;
+    pair[2 * n + 1] = dm_bits;
+  }
+}
+
 cudaError_t launch_quantize(const float* W, int64_t N, int64_t K, int fmt, void* codes,
                             uint16_t* scale, uint16_t* zero, cudaStream_t stream) {
+  if (fmt == 4) {  // int4h: one warp per row
+    quantize_int4h_kernel<<<(unsigned)((N + 7) / 8), 256, 0, stream>>>(W, N, K, (uint32_t*)codes, scale,
+                                                                      reinterpret_cast<uint8_t*>(zero));
+    return cudaGetLastError();
+  }
   const int64_t tasks = N * (K / kGroup);
   const int64_t blocks = (tasks + 7) / 8;
   if (fmt == 0)

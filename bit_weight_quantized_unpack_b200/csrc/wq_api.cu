@@ -56,7 +56,7 @@ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0;
 constexpr int64_t kMaxK = (int64_t)1 << 20;
 
 int check_shape(int fmt, int64_t N, int64_t K) {
-  if (fmt < WQ_INT4 || fmt > WQ_INT3) return WQ_ERR_ARG;
+  if (fmt < WQ_INT4 || fmt > WQ_INT4H) return WQ_ERR_ARG;
   if (N < 1 || N > INT_MAX || K < 128 || K > kMaxK || K % 128 != 0) return WQ_ERR_SHAPE;
   return WQ_OK;
 }
@@ -64,9 +64,15 @@ int check_shape(int fmt, int64_t N, int64_t K) {
 int check_weights(int fmt, const void* codes, const uint16_t* scale, const uint16_t* zero) {
   if (!codes || !scale) return WQ_ERR_ARG;
   if ((fmt == WQ_TERNARY) != (zero == nullptr)) return WQ_ERR_ARG;
+  if (fmt == WQ_INT4H)  // row pairs read as 4-byte words, index bytes bulk-copied
+    return aligned(codes, 16) && aligned(scale, 4) && aligned(zero, 16) ? WQ_OK : WQ_ERR_ALIGN;
   if (!aligned(codes, 16) || !aligned(scale, 2) || (zero && !aligned(zero, 2))) return WQ_ERR_ALIGN;
   return WQ_OK;
 }
+
+// Hierarchical int4 is served by the streaming kernel only: M rows of X of K values each
+// staged in shared memory, M * K <= kHierMaxMK (with M <= 4).
+constexpr int64_t kHierMaxMK = 92160;
 
 // Fill one SetMat; returns its item count (rows per item = 32 >> lanes_log2).
 int64_t plan_mat(wq::SetMat& m, int fmt, const void* codes, const uint16_t* scale,
@@ -87,9 +93,9 @@ int64_t plan_mat(wq::SetMat& m, int fmt, const void* codes, const uint16_t* scal
   return (N + rows - 1) / rows;
 }
 
-// Streaming kernel for a set (int4 / int2) with M = 1 .. 4 rows of X: needs 16-byte aligned
-// codes, scales, zeros and activations, and activations short enough to stage in shared
-// memory.
+// Streaming kernel for a set (int4 / int2 / ternary / int4h) with M = 1 .. 4 rows of X: needs
+// 16-byte aligned codes, metadata and activations, and activations short enough to stage in
+// shared memory.
 // Failure-detection test hook (wq_debug_arm_timeout): poll bound for the next streaming launch
 // on this thread, with one of its ring slots never filled; 0 = disarmed.
 thread_local uint32_t g_arm_polls = 0;
@@ -100,7 +106,8 @@ int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStrea
   static thread_local wq::StreamParams sp;
   static thread_local wq::StreamDesc sd[wq::kStreamMaxMats];
   for (int i = 0; i < count; ++i) sd[i] = {d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K};
-  const int bits = fmt == WQ_INT4 ? 4 : fmt == WQ_INT2 ? 2 : 1;  // 1: ternary
+  // format tag: 4 / 2 bits, 1 ternary, kStreamHier
+  const int bits = fmt == WQ_INT4 ? 4 : fmt == WQ_INT2 ? 2 : fmt == WQ_INT4H ? wq::kStreamHier : 1;
   const int smem = wq::stream_plan(sp, bits, count, sd, (int)M);
   if (smem == 0) return WQ_OK;
   *done = true;
@@ -112,8 +119,6 @@ int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStrea
   return cuda_status(wq::launch_gemv_stream(sp, bits, (int)M, smem, stream));
 }
 
-// Streaming tensor-core kernel for an int4 set with M = 1 .. 8 rows of X: needs 16-byte
-// aligned codes and activations, and K <= 32768 (activations staged in shared memory).
 // int3 set: one warp per output row (any M).
 int launch_int3(const wq_linear_desc* d, int count, cudaStream_t stream) {
   static thread_local wq::SetParams p;
@@ -179,7 +184,7 @@ namespace wq {
 namespace {
 // The plan of the last argmax_prepare on this thread (consumed by argmax_launch).
 thread_local StreamParams g_am_stream;
-thread_local int g_am_bits = 0;  // 0: no plan; 4 or 2: int4 / int2 on the streaming kernel
+thread_local int g_am_bits = 0;  // 0: no plan; else the streaming kernel's format tag
 thread_local int g_am_smem = 0;
 }  // namespace
 
@@ -190,12 +195,12 @@ int argmax_prepare(const uint16_t* x, const void* codes, const uint16_t* scale, 
   if (st != WQ_OK) return st;
   if (fmt == WQ_TERNARY || fmt == WQ_INT3 || !x || !argmax) return WQ_ERR_ARG;
   if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
-  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scale, 16) || !aligned(zero, 16) ||
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scale, fmt == WQ_INT4H ? 4 : 16) || !aligned(zero, 16) ||
       (y && !aligned(y, 2)) || !aligned(argmax, 4))
     return WQ_ERR_ALIGN;
   if (K > 32768) return WQ_ERR_SHAPE;
   if ((st = check_device()) != WQ_OK) return st;
-  const int bits = fmt == WQ_INT4 ? 4 : 2;
+  const int bits = fmt == WQ_INT4 ? 4 : fmt == WQ_INT4H ? kStreamHier : 2;
   const StreamDesc d = {codes, scale, zero, x, y, N, K};
   g_am_smem = stream_plan(g_am_stream, bits, 1, &d, 1);
   if (g_am_smem == 0) return WQ_ERR_SHAPE;
@@ -219,7 +224,7 @@ extern "C" {
 
 size_t wq_codes_bytes(int fmt, int64_t N, int64_t K) {
   if (check_shape(fmt, N, K) != WQ_OK) return 0;
-  if (fmt == WQ_INT4) return (size_t)(N * K / 2);
+  if (fmt == WQ_INT4 || fmt == WQ_INT4H) return (size_t)(N * K / 2);
   if (fmt == WQ_INT2) return (size_t)(N * K / 4);
   if (fmt == WQ_INT3) return (size_t)(N * K * 3 / 8);
   return (size_t)(N * 26 * (K / 128));
@@ -230,11 +235,21 @@ size_t wq_meta_count(int64_t N, int64_t K) {
   return (size_t)(N * (K / 128));
 }
 
+size_t wq_scale_bytes(int fmt, int64_t N, int64_t K) {
+  if (check_shape(fmt, N, K) != WQ_OK) return 0;
+  return fmt == WQ_INT4H ? (size_t)(4 * N) : (size_t)(2 * N * (K / 128));
+}
+
+size_t wq_zero_bytes(int fmt, int64_t N, int64_t K) {
+  if (check_shape(fmt, N, K) != WQ_OK || fmt == WQ_TERNARY) return 0;
+  return fmt == WQ_INT4H ? (size_t)(N * (K / 32)) : (size_t)(2 * N * (K / 128));
+}
+
 int wq_quantize(const float* W, int64_t N, int64_t K, int fmt, int group, void* codes,
                 uint16_t* scale, uint16_t* zero, void* stream) {
   int st = check_shape(fmt, N, K);
   if (st != WQ_OK) return st;
-  if (group != 128 || !W) return WQ_ERR_ARG;
+  if (group != (fmt == WQ_INT4H ? 32 : 128) || !W) return WQ_ERR_ARG;
   if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
   if (!aligned(W, 16)) return WQ_ERR_ALIGN;
   if ((st = check_device()) != WQ_OK) return st;
@@ -250,6 +265,13 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
   if ((st = check_weights(fmt, codes, scale, zero)) != WQ_OK) return st;
   if (!aligned(X, 16) || !aligned(Y, 2)) return WQ_ERR_ALIGN;
   if ((st = check_device()) != WQ_OK) return st;
+  if (fmt == WQ_INT4H) {
+    if (M > wq::kStreamMaxRows || M * K > kHierMaxMK) return WQ_ERR_UNSUPPORTED;
+    const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, M};
+    bool done = false;
+    const int r = try_stream(fmt, 1, &d, M, (cudaStream_t)stream, &done);
+    return done ? r : WQ_ERR_UNSUPPORTED;
+  }
   if (fmt == WQ_INT3) {
     const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, M};
     return launch_int3(&d, 1, (cudaStream_t)stream);
@@ -300,7 +322,7 @@ int wq_gemv(const uint16_t* x, const void* codes, const uint16_t* scale, const u
 
 int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream) {
   if (!descs || count < 1 || count > WQ_LINEAR_SET_MAX) return WQ_ERR_ARG;
-  if (fmt < WQ_INT4 || fmt > WQ_INT3) return WQ_ERR_ARG;
+  if (fmt < WQ_INT4 || fmt > WQ_INT4H) return WQ_ERR_ARG;
   static_assert(WQ_LINEAR_SET_MAX == wq::kSetMax, "set size");
   static thread_local wq::SetParams p;
   p.count = count;
@@ -323,6 +345,14 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
   }
   int st0 = check_device();
   if (st0 != WQ_OK) return st0;
+  if (fmt == WQ_INT4H) {
+    if (M > wq::kStreamMaxRows) return WQ_ERR_UNSUPPORTED;
+    for (int i = 0; i < count; ++i)
+      if (M * descs[i].K > kHierMaxMK) return WQ_ERR_UNSUPPORTED;
+    bool done = false;
+    const int r = try_stream(fmt, count, descs, M, (cudaStream_t)stream, &done);
+    return done ? r : WQ_ERR_UNSUPPORTED;
+  }
   if (fmt == WQ_INT3) return launch_int3(descs, count, (cudaStream_t)stream);
   {
     bool done = false;
@@ -415,7 +445,9 @@ const char* wq_status_str(int status) {
     case WQ_ERR_SHAPE: return "WQ_ERR_SHAPE: N, K or M outside the supported range";
     case WQ_ERR_ALIGN: return "WQ_ERR_ALIGN: pointer not aligned as required";
     case WQ_ERR_CUDA: return "WQ_ERR_CUDA: a CUDA call or launch failed";
-    case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+    case WQ_ERR_UNSUPPORTED:
+      return "WQ_ERR_UNSUPPORTED: not served here (needs an sm_100 (B200) device; WQ_INT4H needs M <= 4 and "
+             "M * K <= 92160)";
     case WQ_ERR_SCRATCH: return "WQ_ERR_SCRATCH: the launch needs more scratch than the library's static array holds";
     default: return "unknown wq_status";
   }

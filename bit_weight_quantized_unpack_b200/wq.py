@@ -20,8 +20,8 @@ if not os.path.exists(_LIB_PATH):
                       "`python -m bit_weight_quantized_unpack_b200.build`")
 _lib = ctypes.CDLL(_LIB_PATH)
 
-WQ_INT4, WQ_INT2, WQ_TERNARY, WQ_INT3 = 0, 1, 2, 3
-FMT = {"int4": WQ_INT4, "int2": WQ_INT2, "ternary": WQ_TERNARY, "int3": WQ_INT3}
+WQ_INT4, WQ_INT2, WQ_TERNARY, WQ_INT3, WQ_INT4H = 0, 1, 2, 3, 4
+FMT = {"int4": WQ_INT4, "int2": WQ_INT2, "ternary": WQ_TERNARY, "int3": WQ_INT3, "int4h": WQ_INT4H}
 WQ_OK, WQ_ERR_ARG, WQ_ERR_SHAPE, WQ_ERR_ALIGN, WQ_ERR_CUDA, WQ_ERR_UNSUPPORTED, WQ_ERR_SCRATCH = range(7)
 WQ_ARGMAX_STATIC_SCRATCH_BYTES = 16384
 WQ_LINEAR_SET_MAX = 256
@@ -38,6 +38,8 @@ class wq_linear_desc(ctypes.Structure):
 _sig = {
     "wq_codes_bytes": (ctypes.c_size_t, [_i, _i64, _i64]),
     "wq_meta_count": (ctypes.c_size_t, [_i64, _i64]),
+    "wq_scale_bytes": (ctypes.c_size_t, [_i, _i64, _i64]),
+    "wq_zero_bytes": (ctypes.c_size_t, [_i, _i64, _i64]),
     "wq_quantize": (_i, [_p, _i64, _i64, _i, _i, _p, _p, _p, _p]),
     "wq_gemv": (_i, [_p, _p, _p, _p, _i, _i64, _i64, _p, _p]),
     "wq_gemm": (_i, [_p, _i64, _p, _p, _p, _i, _i64, _i64, _p, _p]),
@@ -98,6 +100,14 @@ def wq_codes_bytes(fmt, N: int, K: int) -> int:
 
 def wq_meta_count(N: int, K: int) -> int:
     return _lib.wq_meta_count(N, K)
+
+
+def wq_scale_bytes(fmt, N: int, K: int) -> int:
+    return _lib.wq_scale_bytes(_fmt(fmt), N, K)
+
+
+def wq_zero_bytes(fmt, N: int, K: int) -> int:
+    return _lib.wq_zero_bytes(_fmt(fmt), N, K)
 
 
 def wq_quantize(W, N, K, fmt, group, codes, scale, zero, stream=None) -> None:
@@ -189,13 +199,20 @@ def wq_debug_arm_timeout(polls: int) -> None:
 # ---- allocation helpers (torch owns the memory) ------------------------------------
 
 def alloc_packed(N: int, K: int, fmt, device="cuda"):
-    """Empty (codes, scale, zero) tensors for an [N, K] weight; zero is None for ternary."""
+    """Empty (codes, scale, zero) tensors for an [N, K] weight; zero is None for ternary.
+    scale holds fp16 bits (int16); zero too, except for int4h, whose zero is the index bytes
+    (uint8 [N * K / 32]) and whose scale is the row pairs (int16 [2 N])."""
     f = _fmt(fmt)
     nbytes = wq_codes_bytes(f, N, K)
     if nbytes == 0:
         raise WQError(WQ_ERR_SHAPE, "alloc_packed")
     codes = torch.empty(nbytes, dtype=torch.uint8, device=device)
-    meta = wq_meta_count(N, K)
-    scale = torch.empty(meta, dtype=torch.int16, device=device)
-    zero = None if f == WQ_TERNARY else torch.empty(meta, dtype=torch.int16, device=device)
+    scale = torch.empty(wq_scale_bytes(f, N, K) // 2, dtype=torch.int16, device=device)
+    zb = wq_zero_bytes(f, N, K)
+    if f == WQ_TERNARY:
+        zero = None
+    elif f == WQ_INT4H:
+        zero = torch.empty(zb, dtype=torch.uint8, device=device)
+    else:
+        zero = torch.empty(zb // 2, dtype=torch.int16, device=device)
     return codes, scale, zero

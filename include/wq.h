@@ -12,6 +12,11 @@
  *   - WQ_TERNARY: trits t in {-1, 0, +1} with one fp16 absmean scale per group,
  *     w_hat = t * s, five trits per byte in base 3 (format table row "ternary g128";
  *     TKintegers K5, "What is K5?": five balanced-ternary digits make a one-byte code).
+ *   - WQ_INT4H: hierarchical int4 in groups of 32: 4-bit codes q in [0, 15]; per group g
+ *     two 4-bit indices a_g, b_g; per row one fp16 pair (d, dm);
+ *     w_hat = (d a_g) q - (dm b_g) (Whetstone README, "What the weights can actually
+ *     survive": two 4-bit indices per group of 32 against an f16 pair per row, the GGUF
+ *     Q4_K idea of "Prior art"; format table row "int4 hier-g32", 4.28 bits/weight).
  * Products accumulate in fp32; y is rounded to fp16 once, to nearest-even.
  * Batch-1 decode is bound by memory bandwidth (Whetstone README, "The one fact that
  * shapes everything": tok/s ceiling = bandwidth / bytes read per token), so the
@@ -24,6 +29,13 @@
  *            z = clamp(rint(-lo / s), 0, Q),  q = clamp(rint(w / s) + z, 0, Q)
  *   ternary: a = (|w_0| + |w_1| + ... + |w_127|) / 128, summed left to right
  *            s = fp16_rne(a), s := 1 if s == 0,  t = clamp(rint(w / s), -1, 1)
+ *   int4h (per row; groups of 32):
+ *            per group: lo = min w, hi = max w, m_g = max(0, -lo), s_g = (hi + m_g) / 15
+ *            d = rs(max_g s_g), dm = rs(max_g m_g), where rs(v) = fp16_rne(v / 15), except
+ *            rs(0) = 1 and rs(v) = 2^-24 (smallest positive binary16) if v > 0 rounds to 0
+ *            (Whetstone README, "New in 0.6.0": the shared row scale must not underflow)
+ *            a_g = clamp(rint(s_g / d), 0, 15), b_g = clamp(rint(m_g / dm), 0, 15)
+ *            S = d a_g, Z = dm b_g (exact), q = clamp(rint((w + Z) / S), 0, 15), q = 0 if S == 0
  * fp16_rne is the direct float64 -> binary16 rounding (never through float32).
  * Inputs must be finite.
  *
@@ -41,6 +53,10 @@
  *   scale, zero  fp16 bits (uint16) [N, G]; zero is unused (NULL) for WQ_TERNARY; a zero
  *                point is an integer in [0, 2^b - 1] (as wq_quantize writes it); the
  *                kernels use its nearest integer
+ *   int4h        codes as int4 (uint32 [N, K/8]); `scale` is the row pair, fp16 bits
+ *                uint16 [N, 2] = (d, dm); `zero` points to the index BYTES, uint8
+ *                [N, K/32], byte g of a row = a_g | b_g << 4 (passed through the
+ *                uint16_t* parameter); scale 4-byte and zero 16-byte aligned
  *   x, X, y, Y   fp16 bits (uint16), X [M, K] and Y [M, N] row-major
  *
  * Conventions.
@@ -65,7 +81,7 @@
 extern "C" {
 #endif
 
-typedef enum { WQ_INT4 = 0, WQ_INT2 = 1, WQ_TERNARY = 2, WQ_INT3 = 3 } wq_fmt;
+typedef enum { WQ_INT4 = 0, WQ_INT2 = 1, WQ_TERNARY = 2, WQ_INT3 = 3, WQ_INT4H = 4 } wq_fmt;
 
 typedef enum {
   WQ_OK = 0,
@@ -73,21 +89,30 @@ typedef enum {
   WQ_ERR_SHAPE = 2,        /* N, K or M outside the supported range, K % 128 != 0 */
   WQ_ERR_ALIGN = 3,        /* a pointer is not aligned as required above */
   WQ_ERR_CUDA = 4,         /* a CUDA call or launch failed (see wq_last_cuda_error) */
-  WQ_ERR_UNSUPPORTED = 5,  /* valid request the library cannot serve here (e.g. no sm_100 GPU) */
+  WQ_ERR_UNSUPPORTED = 5,  /* valid request the library cannot serve here (no sm_100 GPU, or
+                              WQ_INT4H outside its product range, see wq_gemm) */
   WQ_ERR_SCRATCH = 6       /* needs more scratch than the library's static array holds */
 } wq_status;
 
 /* Bytes of packed codes for an [N, K] weight in format fmt (0 on invalid arguments):
- * int4 N*K/2, int3 N*K*3/8, int2 N*K/4, ternary N*26*(K/128). */
+ * int4 and int4h N*K/2, int3 N*K*3/8, int2 N*K/4, ternary N*26*(K/128). */
 size_t wq_codes_bytes(int fmt, int64_t N, int64_t K);
 
-/* Number of fp16 entries of the scale array (and of the zero array): N * K / 128. */
+/* Number of fp16 entries of the scale array (and of the zero array) of the g128 formats:
+ * N * K / 128. */
 size_t wq_meta_count(int64_t N, int64_t K);
 
+/* Bytes of the scale and of the zero array of an [N, K] weight in format fmt (0 on invalid
+ * arguments, and wq_zero_bytes is 0 for WQ_TERNARY): 2 N K / 128 each for the g128 formats;
+ * int4h 4 N (the row pairs) and N K / 32 (the index bytes). */
+size_t wq_scale_bytes(int fmt, int64_t N, int64_t K);
+size_t wq_zero_bytes(int fmt, int64_t N, int64_t K);
+
 /* Quantise W (fp32 [N, K], device) into codes / scale / zero as defined above.
- * group must be 128. zero must be NULL for WQ_TERNARY and non-NULL otherwise.
- * Whetstone README, "What the weights can actually survive" (round-to-nearest group
- * quantisation) and TKintegers K5, "What is K5?" (base-3 trit bytes). */
+ * group must be 128 (32 for WQ_INT4H). zero must be NULL for WQ_TERNARY and non-NULL
+ * otherwise. Whetstone README, "What the weights can actually survive" (round-to-nearest
+ * group quantisation, hierarchical group-32 metadata) and TKintegers K5, "What is K5?"
+ * (base-3 trit bytes). */
 int wq_quantize(const float* W, int64_t N, int64_t K, int fmt, int group,
                 void* codes, uint16_t* scale, uint16_t* zero, void* stream);
 
@@ -99,6 +124,8 @@ int wq_gemv(const uint16_t* x, const void* codes, const uint16_t* scale,
             void* stream);
 
 /* Y[m, n] = fp16( sum_k X[m, k] * w_hat[n, k] ) for M activation rows, 1 <= M <= 2048.
+ * WQ_INT4H (a decode format) is served for M <= 4 and M * K <= 92160 only, with codes, zero
+ * and X 16-byte aligned; other M or K give WQ_ERR_UNSUPPORTED (before any launch).
  * M = 1 runs the wq_gemv kernel. Small M streams the weights once and reuses each
  * dequantised weight for every row of X (int4 with 2 <= M <= 32: warp-level tensor-core
  * MMAs fed from registers); large M dequantises weight tiles into shared memory as fp16
@@ -144,15 +171,16 @@ size_t wq_argmax_workspace_bytes(void);
  * as fp16 values, ties to the lowest n -- in one launch, with no read-back of y (Whetstone
  * README, notes on --temperature 0: greedy decoding stays on the GPU because the argmax is
  * written where the next step reads it).
- *   fmt        WQ_INT4 or WQ_INT2 (WQ_ERR_ARG otherwise).
+ *   fmt        WQ_INT4, WQ_INT2 or WQ_INT4H (WQ_ERR_ARG otherwise).
  *   y          device fp16 [N], or NULL to skip storing the outputs.
  *   argmax     device int32, written with the row index.
  *   workspace  device buffer of at least wq_argmax_workspace_bytes() bytes, 16-byte aligned,
  *              zero-filled by the caller before its first use; every call leaves its first
  *              4 bytes zero again. Two calls that share a work space must not overlap on the
  *              GPU (same stream, or ordered by events).
- * codes, scale, zero and x must be 16-byte aligned (WQ_ERR_ALIGN) and K at most 32768
- * (WQ_ERR_SHAPE); other requirements as for wq_gemv. Inputs must be finite. */
+ * codes, scale, zero and x must be 16-byte aligned (WQ_ERR_ALIGN; for WQ_INT4H scale 4-byte)
+ * and K at most 32768 (WQ_ERR_SHAPE); other requirements as for wq_gemv. Inputs must be
+ * finite. */
 int wq_gemv_argmax(const uint16_t* x, const void* codes, const uint16_t* scale,
                    const uint16_t* zero, int fmt, int64_t N, int64_t K, uint16_t* y,
                    int32_t* argmax, void* workspace, size_t workspace_bytes, void* stream);

@@ -53,8 +53,24 @@ def test_sizes(lib):
         tot = lib.wq_codes_bytes(fmt, 64, 1024) + 2 * meta_arrays * lib.wq_meta_count(64, 1024)
         assert tot * 8 / (64 * 1024) == bpw
     assert lib.wq_codes_bytes(0, 4, 100) == 0      # K not a multiple of 128
-    assert lib.wq_codes_bytes(4, 4, 128) == 0      # unknown format
+    assert lib.wq_codes_bytes(5, 4, 128) == 0      # unknown format
     assert lib.wq_codes_bytes(0, 0, 128) == 0
+    # int4h: int4 codes + one index byte per 32 weights + one fp16 pair per row; the stored
+    # bits per weight are 4 + 8/32 + 32/K (the Whetstone README format table's 4.28 is the
+    # whole-model figure, pinned in the oracle tests)
+    for f in ("wq_scale_bytes", "wq_zero_bytes"):
+        getattr(lib, f).restype = ctypes.c_size_t
+        getattr(lib, f).argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64]
+    N, K = 151936, 896
+    assert lib.wq_codes_bytes(4, N, K) == N * K // 2
+    assert lib.wq_scale_bytes(4, N, K) == 4 * N
+    assert lib.wq_zero_bytes(4, N, K) == N * K // 32
+    tot = lib.wq_codes_bytes(4, N, K) + lib.wq_scale_bytes(4, N, K) + lib.wq_zero_bytes(4, N, K)
+    assert tot * 8 / (N * K) == pytest.approx(4 + 8 / 32 + 32 / K, rel=1e-12)
+    for fmt in (0, 1, 3):
+        assert lib.wq_scale_bytes(fmt, N, K) == lib.wq_zero_bytes(fmt, N, K) == 2 * N * 7
+    assert lib.wq_scale_bytes(2, N, K) == 2 * N * 7 and lib.wq_zero_bytes(2, N, K) == 0
+    assert lib.wq_scale_bytes(5, N, K) == 0 and lib.wq_zero_bytes(4, N, 100) == 0
 
 
 def test_argument_checks_reject_before_any_launch(lib):
@@ -78,6 +94,11 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert wq._lib.wq_gemv(P, P + 4, P, P, 0, 8, 128, P, S) == wq.WQ_ERR_ALIGN
     assert wq._lib.wq_gemv(P, P, P + 1, P, 0, 8, 128, P, S) == wq.WQ_ERR_ALIGN
     assert wq._lib.wq_quantize(P + 4, 8, 128, 0, 128, P, P, P, S) == wq.WQ_ERR_ALIGN
+    # int4h: group 32, row pairs 4-byte and index bytes 16-byte aligned
+    assert wq._lib.wq_quantize(P, 8, 128, 4, 128, P, P, P, S) == wq.WQ_ERR_ARG
+    assert wq._lib.wq_gemv(P, P, P + 2, P, 4, 8, 128, P, S) == wq.WQ_ERR_ALIGN
+    assert wq._lib.wq_gemv(P, P, P, P + 4, 4, 8, 128, P, S) == wq.WQ_ERR_ALIGN
+    assert wq._lib.wq_gemv(P, P, P, None, 4, 8, 128, P, S) == wq.WQ_ERR_ARG
     # linear set: count range, and a bad entry anywhere rejects the whole call
     good = (P, P, P, P, P, 8, 128)
     arr = wq.make_linear_set([good, (P, P, P, P, P, 8, 130)])
