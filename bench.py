@@ -34,8 +34,12 @@ from bit_weight_quantized_unpack_b200 import synth, workloads  # noqa: E402
 METRIC = "int4 g128 batch-1 GEMV weight GB/s (% of HBM peak); M=512 GEMM TFLOPS"
 INT4_BYTES_PER_WEIGHT = 0.5 + 4 / 128  # codes + fp16 scale + fp16 zero per 128 weights
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gemv_stream_kernel launch
-# over the 0.5B decode set, from one ncu capture of the current kernel (None once it changes)
-GEMV_TRAFFIC_BYTES = 263553280 + 5531648
+# over the 0.5B decode set, from one ncu capture of the kernel as it is now (None when the
+# kernel changed after the capture); TRAFFIC_SOURCE names that capture
+GEMV_TRAFFIC_BYTES = 263556352 + 3634432
+TRAFFIC_SOURCE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
+                  "-k regex:gemv_stream -s 10 -c 1 python bench.py --steps 20 --warmup 5 --no-rows --quick")
+L2_BYTES = 126 * 1000 * 1000
 
 
 def peaks():
@@ -187,6 +191,39 @@ def time_steps(step, steps, warmup, ws, clocks=None):
     return ev0.elapsed_time(ev1) / steps  # ms per step on this rank
 
 
+def step_stats(step, n, warm=3):
+    """Per-step device times from one CUDA event between consecutive steps on the launching
+    stream: median, p10 and p90 in ms (the pages' timing hygiene: median with p10 / p90)."""
+    for i in range(warm):
+        step(i)
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    evs[0].record()
+    for i in range(n):
+        step(i)
+        evs[i + 1].record()
+    torch.cuda.synchronize()
+    d = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(n))
+
+    def q(f):
+        return d[min(n - 1, int(f * (n - 1) + 0.5))]
+    return {"median_ms": q(0.5), "p10_ms": q(0.1), "p90_ms": q(0.9), "n": n}
+
+
+def graph_of(calls):
+    """A CUDA graph replaying `calls` (each enqueues work on torch's current stream); every
+    call runs once before capture, so that the library's one-time set-up is done."""
+    for f in calls:
+        f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in calls:
+            f()
+    torch.cuda.synchronize()
+    return g
+
+
 class _Null:
     def __enter__(self):
         return self
@@ -263,9 +300,68 @@ def bench_rows(args, pk):
         del copies
         torch.cuda.empty_cache()
     rows.update(bench_int4h_set(args, pk))
+    rows.update(bench_config0(args, pk))
+    rows.update(bench_per_matrix_graphs(args, pk))
     rows.update(bench_batch_sweep(args, pk))
     rows.update(bench_7b_set(args, pk))
     return rows
+
+
+def bench_config0(args, pk):
+    """The single 896 x 896 int4 matrix at batch 1, one wq_gemv per product, over enough
+    copies (C) that one pass reads 3 x L2 from HBM. The launches of one pass are replayed as a
+    CUDA graph (back to back on the GPU, no host gaps): per launch = pass / C."""
+    from bit_weight_quantized_unpack_b200 import wq
+    wl = workloads.WORKLOADS[0]
+    N = K = 896
+    nb = wq.wq_codes_bytes("int4", N, K) + wq.wq_scale_bytes("int4", N, K) + wq.wq_zero_bytes("int4", N, K)
+    copies = 3 * L2_BYTES // nb + 1
+    W = synth.weights(N, K, wl["sigma"], wl["seed"], device="cuda")
+    c0, s0, z0 = wq.alloc_packed(N, K, "int4")
+    wq.wq_quantize(W, N, K, "int4", 128, c0, s0, z0)
+    C = c0.repeat(copies, 1) if c0.dim() == 2 else c0.view(1, -1).repeat(copies, 1)
+    S = s0.view(1, -1).repeat(copies, 1)
+    Z = z0.view(1, -1).repeat(copies, 1)
+    x = synth.activations(1, K, synth.sub_seed(wl["seed"], 0, 1), device="cuda")[0]
+    y = torch.empty(N, dtype=torch.float16, device="cuda")
+    g = graph_of([lambda i=i: wq.wq_gemv(x, C[i], S[i], Z[i], "int4", N, K, y) for i in range(copies)])
+    st = step_stats(lambda i: g.replay(), 20 if not args.quick else 5)
+    per = st["median_ms"] / copies
+    out = {"gemv_single_896_int4": {"us_per_launch": per * 1e3, "p10_us": st["p10_ms"] / copies * 1e3,
+                                    "p90_us": st["p90_ms"] / copies * 1e3, "GBps": nb / per / 1e6,
+                                    "frac_hbm": nb / per / 1e6 / pk["hbm_gbs"], "copies": copies,
+                                    "bytes_per_pass": nb * copies,
+                                    "launch": "CUDA graph of one wq_gemv per copy"}}
+    del C, S, Z, g
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_per_matrix_graphs(args, pk):
+    """One token of the 0.5B set (2 copies) and of the 7B set as a CUDA graph of one wq_gemv per
+    matrix, beside the one-launch wq_linear_set (Whetstone README, "The baseline, and where the
+    opportunity actually is": dispatch and launch overhead set the baseline's speed)."""
+    from bit_weight_quantized_unpack_b200 import wq
+    out = {}
+    for widx, copies, name in ((1, 2, "qwen05b"), (3, 1, "qwen7b")):
+        sets, weights, _, _ = build_set(widx, copies=copies)
+        nbytes = weights * INT4_BYTES_PER_WEIGHT
+        calls = [lambda e=e: wq.wq_gemv(e[3], e[0], e[1], e[2], "int4", e[5], e[6], e[4])
+                 for st in sets for e in st["ent"]]
+        g = graph_of(calls)
+        gs = step_stats(lambda i: g.replay(), 20 if not args.quick else 5)
+        ls = step_stats(lambda i: wq.wq_linear_set(sets[i % copies]["desc"], sets[0]["count"], "int4"),
+                        100 if not args.quick else 10)
+        per_tok_graph = gs["median_ms"] / copies
+        out[f"per_matrix_graph_{name}_int4"] = {
+            "ms_per_token": per_tok_graph, "GBps": nbytes / per_tok_graph / 1e6,
+            "launches_per_token": len(calls) // copies,
+            "grouped_ms_per_token": ls["median_ms"], "grouped_GBps": nbytes / ls["median_ms"] / 1e6,
+            "grouped_p10_ms": ls["p10_ms"], "grouped_p90_ms": ls["p90_ms"],
+            "speedup_grouped_vs_graph": per_tok_graph / ls["median_ms"]}
+        del sets, g, calls
+        torch.cuda.empty_cache()
+    return out
 
 
 def bench_int4h_set(args, pk):
@@ -377,6 +473,8 @@ def run_ours(args):
 
     e2e_steps = max(args.steps // 4, 10)
     ms_e2e = max_over_ranks(time_steps(step_e2e, e2e_steps, args.warmup, ws), ws)
+    # per-launch spread of the same step (event between consecutive launches)
+    launch_stats = step_stats(step, min(args.steps, 2000))
 
     rows = bench_rows(args, pk) if (rank == 0 and ws == 1 and not args.no_rows) else {}
 
@@ -393,17 +491,21 @@ def run_ours(args):
                        "l2": "inputs larger than L2: 2 rotating copies of the set (525 MB)",
                        "parallelism": f"replicas x{ws}"},
             "implied_tok_s": round(1e3 / ms_max, 1),
+            "launch_stats": {k: (round(v, 5) if isinstance(v, float) else v) for k, v in launch_stats.items()},
             "frac_of_hbm_peak": round(gbs / ws / pk["hbm_gbs"], 4),
             "roofline": {"bound": "hbm", "achieved": round(nbytes / ms / 1e6, 2),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(nbytes / ms / 1e6 / pk["hbm_gbs"], 4),
-                         "traffic": GEMV_TRAFFIC_BYTES, "kernel": "gemv_stream_kernel<4, 256>",
-                         "peak_source": pk["source"]},
+                         "traffic": GEMV_TRAFFIC_BYTES, "traffic_source": TRAFFIC_SOURCE,
+                         "kernel": "gemv_stream_kernel<4, 256>", "peak_source": pk["source"]},
             "e2e": {"value": round(job_gbs(nbytes, ms_e2e, ws), 2), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * K_tot, "d2h_bytes_per_step": 2 * N_tot},
             "gpu_launches": args.steps,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
+            "gemm_m512_tflops": (round(rows["gemm_set_M512"]["TFLOPS"], 1) if "gemm_set_M512" in rows else None),
+            "gemm_m512_frac_of_tensor_peak": (round(rows["gemm_set_M512"]["frac_tensor"], 4)
+                                              if "gemm_set_M512" in rows else None),
             "gemm_m512": ({"TFLOPS": round(rows["gemm_set_M512"]["TFLOPS"], 1),
                            "frac_of_tensor_peak": round(rows["gemm_set_M512"]["frac_tensor"], 4),
                            "peak_tflops": pk["bf16_tflops"],
@@ -438,11 +540,18 @@ def _oracle_sample(rows_div=64):
 
 
 def _threads():
+    """Threads of the BLAS pool the oracle's float64 matrix product runs on (its
+    dequantisation is single-threaded numpy)."""
     try:
         from threadpoolctl import threadpool_info
         return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
     except Exception:
         return 1
+
+
+def _cpu_fields():
+    return {"cores": _threads(), "host_cores": os.cpu_count(),
+            "parallel": "float64 matrix product on the BLAS pool (cores); dequantisation single-threaded"}
 
 
 def cpu_baseline(args):
@@ -458,7 +567,7 @@ def cpu_baseline(args):
             break
     dt = (time.perf_counter() - t0) / reps
     return {"value": round(weights * INT4_BYTES_PER_WEIGHT / dt / 1e9, 4), "unit": "GB/s",
-            "cores": _threads(), "kind": "oracle",
+            **_cpu_fields(), "kind": "oracle",
             "sample": f"every {256 if args.quick else 64}th row of each of the 169 matrices "
                       f"({weights} weights), dequantise + float64 product, {reps} reps"}
 
@@ -469,13 +578,13 @@ def run_reference(args):
     if rank != 0:
         return
     from oracle import wq_oracle as O
-    # size each step's sample so that warmup + steps take about 90 s of host time
+    # size each step's sample so that warmup + steps take about --ref-budget-s of host time
     cal, cal_w = _oracle_sample(1024)
     t0 = time.perf_counter()
     for x, (p, s, z), K in cal:
         O.gemv_packed(x, "int4", p, s, z, K)
     t_cal = time.perf_counter() - t0
-    budget = 90.0 / (args.steps + args.warmup)
+    budget = args.ref_budget_s / (args.steps + args.warmup)
     rows_div = int(min(max(1024 * t_cal / budget, 64), 1 << 20))
     sample, weights = _oracle_sample(rows_div)
     nbytes = weights * INT4_BYTES_PER_WEIGHT
@@ -495,7 +604,7 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": workloads.WORKLOADS[1]["name"],
                                             "sample": f"every {rows_div}th row of each matrix"},
-            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": "GB/s", **_cpu_fields(), "kind": "oracle",
                              "sample": f"every {rows_div}th row of each of the 169 matrices "
                                        f"({weights} weights)"},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -514,6 +623,8 @@ def main():
                     help="time one secondary case alone (for profiling): gemm_set = the "
                          "0.5B set at --batch tokens through wq_linear_set")
     ap.add_argument("--batch", type=int, default=512)
+    ap.add_argument("--ref-budget-s", type=float, default=90.0,
+                    help="host seconds the reference arm's warmup + steps take (about)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

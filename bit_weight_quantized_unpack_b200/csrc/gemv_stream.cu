@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
   }
 
   // ---- producer: the warp's segments, in matrix order, as ring slots (state kept by every
-  // lane alike; lanes 0, 1, 2 issue the codes, scales and zeros copies of a slot together)
+  // lane alike; lane 0 issues the codes and metadata copies of a slot)
   Prod pd;
   pd.cleft = 0;
   pd.pm = mfirst - 1;
@@ -603,13 +603,13 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     const uint32_t units = (uint32_t)(gc & ~(16 / F::MB0 - 1));  // cells in whole units
     const uint32_t mb0 = F::MB0 * units, mb1 = F::MB1 * units;
     const uint32_t cbb = (uint32_t)cb & ~15u;
-    if (!(skip_first && issued == 0)) {
-      if (lane == 0) tc::mbar_arrive_expect_tx(bar, cbb + mb0 + mb1);
-      if (lane == 0 || (lane == 1 && mb0) || (F::MB1 && lane == 2 && mb1)) {
-        const void* src = lane == 0 ? (const void*)pd.c : lane == 1 ? (const void*)pd.m0 : (const void*)pd.m1;
-        const uint32_t d = lane == 0 ? dst : lane == 1 ? dst + F::SC : dst + F::SC + F::META0;
-        bulk_g2s(d, src, lane == 0 ? cbb : lane == 1 ? mb0 : mb1, bar);
-      }
+    // one lane issues the slot's copies: their operands live in uniform registers, so copies
+    // with different operands from several lanes would be issued one lane at a time anyway
+    if (lane == 0 && !(skip_first && issued == 0)) {
+      tc::mbar_arrive_expect_tx(bar, cbb + mb0 + mb1);
+      bulk_g2s(dst, pd.c, cbb, bar);
+      if (mb0) bulk_g2s(dst + F::SC, pd.m0, mb0, bar);
+      if (F::MB1 && mb1) bulk_g2s(dst + F::SC + F::META0, pd.m1, mb1, bar);
     }
     pd.c += cb;
     pd.m0 += F::MB0 * gc;

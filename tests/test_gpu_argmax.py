@@ -86,3 +86,29 @@ def test_argmax_rejects_bad_arguments():
     c3, s3, _ = quantize_gpu(W.cuda(), "ternary")
     with pytest.raises(wq().WQError):                     # ternary is not served
         wq().wq_gemv_argmax(x, c3, s3, None, "ternary", N, K, None, am, ws, nb)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "int2", "int4h"])
+def test_argmax_all_outputs_minus_infinity(fmt):
+    """Finite inputs whose products overflow fp16 to -inf in every row: the pick is still a
+    valid row, the lowest one (all values tie)."""
+    lib = wq()
+    N, K = 300, 128
+    codes, scale, zero = lib.alloc_packed(N, K, fmt)
+    codes.zero_()  # every code 0
+    if fmt == "int4h":
+        # w_hat = d a q - dm b: q = 0, dm = 1000, b = 15 -> -15000 per weight
+        pair = torch.tensor([0x3C00, 0x63D0], dtype=torch.int32).to(torch.int16).repeat(N)
+        scale.copy_(pair.cuda())
+        zero.fill_(0xF1)  # index byte: a = 1, b = 15
+    else:
+        scale.fill_(0x63D0)  # fp16 1000
+        zero.fill_(0x4B80 if fmt == "int4" else 0x4200)  # fp16 15 (int4) / 3 (int2): w_hat < 0
+    x = torch.full((K,), 60000.0, dtype=torch.float16, device="cuda")
+    y = torch.empty(N, dtype=torch.float16, device="cuda")
+    am = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    ws, nb = _workspace()
+    lib.wq_gemv_argmax(x, codes, scale, zero, fmt, N, K, y, am, ws, nb)
+    torch.cuda.synchronize()
+    assert torch.all(torch.isinf(y.float()) & (y.float() < 0)), "every output overflows to -inf"
+    assert int(am.item()) == 0
