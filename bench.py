@@ -210,6 +210,14 @@ def step_stats(step, n, warm=3):
     return {"median_ms": q(0.5), "p10_ms": q(0.1), "p90_ms": q(0.9), "n": n}
 
 
+def row_stats(step, n, nbytes, pk):
+    """A bench row: per-launch median / p10 / p90 (ms) and the median's GB/s of nbytes."""
+    st = step_stats(step, n)
+    gbs = nbytes / st["median_ms"] / 1e6
+    return {"ms": st["median_ms"], "p10_ms": st["p10_ms"], "p90_ms": st["p90_ms"], "GBps": gbs,
+            "frac_hbm": gbs / pk["hbm_gbs"]}
+
+
 def graph_of(calls):
     """A CUDA graph replaying `calls` (each enqueues work on torch's current stream); every
     call runs once before capture, so that the library's one-time set-up is done."""
@@ -238,10 +246,14 @@ def bench_rows(args, pk):
     rows = {}
     N, K = 151936, 896
     wl = workloads.WORKLOADS[2]
-    # lm_head alone, each format; 4+ rotating copies so the working set exceeds L2
+    # lm_head alone, each format; rotating copies of the packed head so that one pass over
+    # them reads at least 3 x L2 from HBM
+    n_launch = 200 if not args.quick else 20
     for fmt in ("int4", "int4h", "int3", "int2", "ternary"):
+        nb = wq.wq_codes_bytes(fmt, N, K) + wq.wq_scale_bytes(fmt, N, K) + wq.wq_zero_bytes(fmt, N, K)
+        n_copies = max(4, -(-3 * L2_BYTES // nb))
         copies = []
-        for cidx in range(6 if fmt != "int4" else 4):
+        for cidx in range(1):
             W = synth.weights_with_outliers(N, K, wl["sigma"], synth.sub_seed(wl["seed"] + cidx, 0, 0),
                                             wl["outlier_frac"], wl["outlier_gain"], device="cuda")
             c, s, z = wq.alloc_packed(N, K, fmt)
@@ -259,16 +271,17 @@ def bench_rows(args, pk):
             wq.wq_quantize(W, N, K, fmt, 32 if fmt == "int4h" else 128, c, s, z)
             del W
             copies.append((c, s, z))
+        # the other copies: the same bytes at other addresses (the stream's cost depends on
+        # where the bytes come from, not on their values)
+        copies += [tuple(None if t is None else t.clone() for t in copies[0]) for _ in range(n_copies - 1)]
         x = synth.activations(1, K, 99, device="cuda")[0]
         y = torch.empty(N, dtype=torch.float16, device="cuda")
-        nb = wq.wq_codes_bytes(fmt, N, K) + wq.wq_scale_bytes(fmt, N, K) + wq.wq_zero_bytes(fmt, N, K)
 
         def step(i, copies=copies, fmt=fmt):
             c, s, z = copies[i % len(copies)]
             wq.wq_gemv(x, c, s, z, fmt, N, K, y)
-        ms = time_steps(step, 200 if not args.quick else 20, 10, 1)
-        rows[f"gemv_lm_head_{fmt}"] = {"ms": ms, "GBps": nb / ms / 1e6,
-                                       "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"]}
+        rows[f"gemv_lm_head_{fmt}"] = {**row_stats(step, n_launch, nb, pk), "copies": n_copies,
+                                       "working_set_MB": n_copies * nb / 1e6}
         if fmt == "int4":
             # fused greedy pick: product and argmax in one launch, y not stored
             ws = torch.zeros(wq.wq_argmax_workspace_bytes(), dtype=torch.uint8, device="cuda")
@@ -277,9 +290,7 @@ def bench_rows(args, pk):
             def step_am(i, copies=copies):
                 c, s, z = copies[i % len(copies)]
                 wq.wq_gemv_argmax(x, c, s, z, "int4", N, K, None, am, ws, ws.numel())
-            ms = time_steps(step_am, 200 if not args.quick else 20, 10, 1)
-            rows["gemv_argmax_lm_head_int4"] = {"ms": ms, "GBps": nb / ms / 1e6,
-                                                "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"]}
+            rows["gemv_argmax_lm_head_int4"] = row_stats(step_am, n_launch, nb, pk)
             # head rescoring: int4 head, top 8 candidates recomputed from an fp16 head copy
             topk = 8
             w16 = synth.weights_with_outliers(N, K, wl["sigma"], synth.sub_seed(wl["seed"], 0, 0),
@@ -292,10 +303,8 @@ def bench_rows(args, pk):
             def step_rs(i, copies=copies):
                 c, s, z = copies[i % len(copies)]
                 wq.wq_gemv_rescore(x, c, s, z, "int4", w16, N, K, topk, y, cand, cl, tok, wsr, wsr.numel())
-            ms = time_steps(step_rs, 200 if not args.quick else 20, 10, 1)
-            rows["gemv_rescore_lm_head_int4"] = {"ms": ms, "GBps": nb / ms / 1e6,
-                                                 "frac_hbm": nb / ms / 1e6 / pk["hbm_gbs"],
-                                                 "topk": topk, "launches": 3}
+            rows["gemv_rescore_lm_head_int4"] = {**row_stats(step_rs, n_launch, nb, pk), "topk": topk,
+                                                 "launches": 3}
             del w16
         del copies
         torch.cuda.empty_cache()
@@ -375,10 +384,8 @@ def bench_int4h_set(args, pk):
     def step(i):
         s = sets[i % len(sets)]
         wq.wq_linear_set(s["desc"], s["count"], "int4h")
-    ms = time_steps(step, 200 if not args.quick else 20, 10, 1)
-    out = {"gemv_set_qwen05b_int4h": {"ms": ms, "GBps": nbytes / ms / 1e6,
-                                      "frac_hbm": nbytes / ms / 1e6 / pk["hbm_gbs"],
-                                      "bytes_per_token": nbytes, "implied_tok_s": 1e3 / ms}}
+    r = row_stats(step, 500 if not args.quick else 20, nbytes, pk)
+    out = {"gemv_set_qwen05b_int4h": {**r, "bytes_per_token": nbytes, "implied_tok_s": 1e3 / r["ms"]}}
     del sets
     torch.cuda.empty_cache()
     return out
@@ -394,10 +401,8 @@ def bench_7b_set(args, pk):
 
     def step(i):
         wq.wq_linear_set(s["desc"], s["count"], "int4")
-    ms = time_steps(step, 20 if not args.quick else 5, 3, 1)
-    out = {"gemv_set_qwen7b_int4": {"ms": ms, "GBps": nbytes / ms / 1e6,
-                                    "frac_hbm": nbytes / ms / 1e6 / pk["hbm_gbs"],
-                                    "implied_tok_s": 1e3 / ms}}
+    r = row_stats(step, 40 if not args.quick else 5, nbytes, pk)
+    out = {"gemv_set_qwen7b_int4": {**r, "implied_tok_s": 1e3 / r["ms"]}}
     del sets, s
     torch.cuda.empty_cache()
     return out
@@ -429,10 +434,12 @@ def bench_batch_sweep(args, pk, Ms=(2, 4, 8, 16, 32, 64, 512, 2048)):
         def one_pass(i, desc=desc):
             wq.wq_linear_set(desc, len(mats), "int4")
         steps = 20 if M >= 512 else 50
-        ms = time_steps(one_pass, steps if not args.quick else 5, 3, 1)
+        st = step_stats(one_pass, steps if not args.quick else 5)
+        ms = st["median_ms"]
         flops = 2.0 * M * weights
         gbs = weights * INT4_BYTES_PER_WEIGHT / ms / 1e6
-        out[f"gemm_set_M{M}"] = {"ms": ms, "TFLOPS": flops / ms / 1e9,
+        out[f"gemm_set_M{M}"] = {"ms": ms, "p10_ms": st["p10_ms"], "p90_ms": st["p90_ms"],
+                                 "TFLOPS": flops / ms / 1e9,
                                  "frac_tensor": flops / ms / 1e9 / pk["bf16_tflops"],
                                  "weight_GBps": gbs, "frac_hbm": gbs / pk["hbm_gbs"],
                                  "kernel": ("gemv_stream_kernel" if M == 1 else

@@ -159,7 +159,10 @@ typedef struct {
  * token reads every weight once, and per-launch overhead dominates small matrices
  * (Whetstone README, "The baseline, and where the opportunity actually is": dispatch and
  * launch overhead, not bytes, set the baseline's speed). All entries must have the same
- * M. 1 <= count <= WQ_LINEAR_SET_MAX; each entry obeys the wq_gemm requirements. */
+ * M. 1 <= count <= WQ_LINEAR_SET_MAX; each entry obeys the wq_gemm requirements. Results equal
+ * the single calls' up to the fp32 summation order of rows whose groups straddle two units of
+ * work (in practice the fp16 outputs are nearly always bit-identical); each call is
+ * deterministic. */
 int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream);
 
 /* Bytes of device work space wq_gemv_argmax needs on the current device (one 8-byte partial
