@@ -626,9 +626,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--quick", action="store_true", help="smaller rows / CPU sample")
     ap.add_argument("--no-rows", action="store_true", help="skip the secondary rows")
-    ap.add_argument("--case", default=None, choices=["gemm_set"],
+    ap.add_argument("--case", default=None, choices=["gemm_set", "int4h_set"],
                     help="time one secondary case alone (for profiling): gemm_set = the "
-                         "0.5B set at --batch tokens through wq_linear_set")
+                         "0.5B set at --batch tokens through wq_linear_set; int4h_set = the "
+                         "0.5B set in hierarchical int4 at batch 1")
     ap.add_argument("--batch", type=int, default=512)
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="host seconds the reference arm's warmup + steps take (about)")
@@ -642,6 +643,11 @@ def main():
         args.quick = False
         r = bench_batch_sweep(args, peaks(), Ms=(args.batch,))
         print(json.dumps({"case": args.case, "batch": args.batch, **r}), flush=True)
+    elif args.case == "int4h_set":
+        torch.cuda.init()
+        args.quick = True
+        r = bench_int4h_set(args, peaks())
+        print(json.dumps({"case": args.case, **r}), flush=True)
     else:
         run_ours(args)
 
