@@ -60,14 +60,14 @@ __host__ __device__ __forceinline__ int xrot(int g) {
   return (BITS == 4 || BITS == HIER) ? (g >> 1) & 3 : BITS == 2 ? (g >> 2) & 1 : 0;
 }
 
-// Per format (BITS = 4, 2, TERN or HIER): bytes of codes per cell (128 weights of a row), ring
+// Per format (BITS = 4, 3, 2, TERN or HIER): bytes of codes per cell (128 weights of a row), ring
 // slot layout (codes, then the per-cell metadata: scales and zeros of the g128 integer
 // formats, scales of ternary, the four index bytes of HIER), staged activation units per group.
 template <int BITS>
 struct Fmt {
   static constexpr bool TRN = BITS == TERN;
   static constexpr bool HR = BITS == HIER;
-  static constexpr int CB = TRN ? 26 : HR ? 64 : 128 * BITS / 8;  // codes bytes per cell: 64 / 32 / 26
+  static constexpr int CB = TRN ? 26 : HR ? 64 : 128 * BITS / 8;  // codes bytes per cell: 64 / 48 / 32 / 26
   static constexpr int CH = TRN ? 1 : CB / 16;          // 16-byte chunks per cell: 4 / 2
   static constexpr int UPC = 16 / CH;                   // activation units per chunk: 4 / 8
   static constexpr int SPS = TRN ? 4 : kStreamSlotCodes / (32 * CB);  // steps of 32 cells per slot
@@ -185,6 +185,53 @@ __device__ __forceinline__ void cell_dot(uint32_t cell, uint32_t xg, uint32_t xs
 #pragma unroll
     for (int m = 0; m < MT; ++m) out[m] = fmaf(a[m][3], 0.015625f, fmaf(a[m][2], 0.0625f, fmaf(a[m][1], 0.25f, a[m][0])));
   }
+}
+
+// int3: out[m] = 2^-24 * sum_k x_mk (q_k - z) over one cell of 48 bytes (12 words, code k at
+// bit 3k; codes 10, 21, 42, ... straddle two words). Codes are taken in pairs (2p, 2p + 1): a
+// funnel shift brings bit 6p to bit 0, a byte permute copies byte 0 to bytes 0 and 2, and one
+// AND leaves code 2p in bits 0-2 (the binary16 subnormal q 2^-24) and code 2p + 1 in bits
+// 19-21 (8 q 2^-24); one packed subtract of (z, 8 z) 2^-24 gives the differences exactly, and
+// the activations pair with them in natural order. The cells of a step sit 48 bytes apart, 12
+// words: the 8 lanes of a shared-memory phase read 8 different bank groups without a permutation.
+template <int MT>
+__device__ __forceinline__ void cell_dot_int3(uint32_t cell, uint32_t xg, uint32_t xs, uint16_t zbits,
+                                              float (&out)[MT]) {
+  uint32_t wd[13];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    const uint4 v = lds128(cell + 16 * c);
+    wd[4 * c] = v.x;
+    wd[4 * c + 1] = v.y;
+    wd[4 * c + 2] = v.z;
+    wd[4 * c + 3] = v.w;
+  }
+  wd[12] = 0u;
+  const uint32_t zi = (uint32_t)__half2int_rn(__ushort_as_half(zbits));
+  const uint32_t zp = zi | (zi << 19);  // (z, 8 z) as binary16 subnormal bits
+  float a[MT][2], b[MT][2];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) a[m][0] = a[m][1] = b[m][0] = b[m][1] = 0.f;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {  // 16 units of 8 activations
+    uint4 xw[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) xw[m] = lds128(xg + m * xs + 16 * u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int bit = 6 * (4 * u + q);
+      const uint32_t w = __funnelshift_r(wd[bit >> 5], wd[(bit >> 5) + 1], bit & 31);
+      const uint32_t d = hsub2_u32(prmt_u32(w, 0u, 0x4040u) & 0x00380007u, zp);  // (q0 - z, 8 (q1 - z))
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint32_t xr = q == 0 ? xw[m].x : q == 1 ? xw[m].y : q == 2 ? xw[m].z : xw[m].w;
+        a[m][q & 1] = fma_f16f16_f32(lo16(d), lo16(xr), a[m][q & 1]);
+        b[m][q & 1] = fma_f16f16_f32(hi16(d), hi16(xr), b[m][q & 1]);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) out[m] = fmaf(b[m][0] + b[m][1], 0.125f, a[m][0] + a[m][1]);
 }
 
 // Ternary: out[m] = 2^-24 * sum_k x_mk t_k over one cell (26 bytes at the 2-byte aligned
@@ -453,6 +500,12 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
           for (int m = 0; m < MT; ++m) v[m] *= sf;
         } else {
         const uint16_t zb = lds16(meta0 + 64 * ss + F::META0);
+        if constexpr (BITS == 3) {
+          cell_dot_int3<MT>(cell0 + 32 * F::CB * ss, xb + 16 * F::XU * gp, xs, zb, v);
+          const float s24 = __half2float(__ushort_as_half(sb)) * 16777216.f;
+#pragma unroll
+          for (int m = 0; m < MT; ++m) v[m] *= s24;
+        } else {
         // chunks in an order permuted by the group index, so that the lanes of one
         // shared-memory phase (consecutive cells) hit different bank groups; the staged
         // activations of each group are stored in that same order (see stage_x), so the
@@ -470,6 +523,7 @@ __device__ __forceinline__ void consume(const Seg& seg, const StreamMat& M, uint
         const float s24 = __half2float(__ushort_as_half(sb)) * 16777216.f;
 #pragma unroll
         for (int m = 0; m < MT; ++m) v[m] *= s24;
+        }
         }
       }
       // segmented inclusive scan over the lanes of each row within this step
@@ -663,7 +717,8 @@ __global__ void __launch_bounds__(T, kStreamMaxCtasPerSm) gemv_stream_kernel(con
     for (int t = threadIdx.x; t < MT * units; t += T) {
       const int m = t / units, u = t - m * units;
       const int g = u >> 4, lc = (u & 15) / F::UPC, i = u & (F::UPC - 1);
-      const int pu = m * rowu + F::XU * g + F::UPC * (lc ^ xrot<BITS>(g)) + i;
+      // int3: natural order (its cells need no chunk permutation)
+      const int pu = BITS == 3 ? m * rowu + F::XU * g + (u & 15) : m * rowu + F::XU * g + F::UPC * (lc ^ xrot<BITS>(g)) + i;
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(xb + 16 * pu), "l"(M.x + (size_t)8 * t)
                    : "memory");
     }
@@ -904,6 +959,7 @@ int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int m
   if (count < 1 || count > kStreamMaxMats || mt < 1 || mt > kStreamMaxRows) return 0;
   switch (bits) {
     case 4: return plan_t<4>(p, count, d, mt);
+    case 3: return plan_t<3>(p, count, d, mt);
     case 2: return plan_t<2>(p, count, d, mt);
     case HIER: return plan_t<HIER>(p, count, d, mt);
     default: return plan_t<TERN>(p, count, d, mt);
@@ -913,6 +969,7 @@ int stream_plan(StreamParams& p, int bits, int count, const StreamDesc* d, int m
 cudaError_t launch_gemv_stream(const StreamParams& p, int bits, int mt, int smem, cudaStream_t stream) {
   switch (bits) {
     case 4: return launch_b<4>(p, mt, smem, stream);
+    case 3: return launch_b<3>(p, mt, smem, stream);
     case 2: return launch_b<2>(p, mt, smem, stream);
     case HIER: return launch_b<HIER>(p, mt, smem, stream);
     default: return launch_b<TERN>(p, mt, smem, stream);

@@ -67,7 +67,7 @@ struct StreamDesc {
   int64_t N, K;
 };
 
-// Format tags of the streaming kernel: bits 4 or 2 (g128 integer codes), 1 (ternary), 5
+// Format tags of the streaming kernel: bits 4, 3 or 2 (g128 integer codes), 1 (ternary), 5
 // (hierarchical int4: codes as int4, `scale` the fp16 row pairs [N, 2], `zero` the index bytes
 // [N, K/32]).
 constexpr int kStreamHier = 5;

@@ -106,8 +106,8 @@ int try_stream(int fmt, int count, const wq_linear_desc* d, int64_t M, cudaStrea
   static thread_local wq::StreamParams sp;
   static thread_local wq::StreamDesc sd[wq::kStreamMaxMats];
   for (int i = 0; i < count; ++i) sd[i] = {d[i].codes, d[i].scale, d[i].zero, d[i].x, d[i].y, d[i].N, d[i].K};
-  // format tag: 4 / 2 bits, 1 ternary, kStreamHier
-  const int bits = fmt == WQ_INT4 ? 4 : fmt == WQ_INT2 ? 2 : fmt == WQ_INT4H ? wq::kStreamHier : 1;
+  // format tag: 4 / 3 / 2 bits, 1 ternary, kStreamHier
+  const int bits = fmt == WQ_INT4 ? 4 : fmt == WQ_INT3 ? 3 : fmt == WQ_INT2 ? 2 : fmt == WQ_INT4H ? wq::kStreamHier : 1;
   const int smem = wq::stream_plan(sp, bits, count, sd, (int)M);
   if (smem == 0) return WQ_OK;
   *done = true;
@@ -272,8 +272,13 @@ int wq_gemm(const uint16_t* X, int64_t M, const void* codes, const uint16_t* sca
     const int r = try_stream(fmt, 1, &d, M, (cudaStream_t)stream, &done);
     return done ? r : WQ_ERR_UNSUPPORTED;
   }
-  if (fmt == WQ_INT3) {
+  if (fmt == WQ_INT3) {  // streaming kernel for M <= 4 where it applies, else one warp per row
     const wq_linear_desc d = {codes, scale, zero, X, Y, N, K, M};
+    if (M <= wq::kStreamMaxRows) {
+      bool done = false;
+      const int r = try_stream(fmt, 1, &d, M, (cudaStream_t)stream, &done);
+      if (done) return r;
+    }
     return launch_int3(&d, 1, (cudaStream_t)stream);
   }
   {
@@ -353,7 +358,14 @@ int wq_linear_set(const wq_linear_desc* descs, int count, int fmt, void* stream)
     const int r = try_stream(fmt, count, descs, M, (cudaStream_t)stream, &done);
     return done ? r : WQ_ERR_UNSUPPORTED;
   }
-  if (fmt == WQ_INT3) return launch_int3(descs, count, (cudaStream_t)stream);
+  if (fmt == WQ_INT3) {
+    if (M <= wq::kStreamMaxRows) {
+      bool done = false;
+      const int r = try_stream(fmt, count, descs, M, (cudaStream_t)stream, &done);
+      if (done) return r;
+    }
+    return launch_int3(descs, count, (cudaStream_t)stream);
+  }
   {
     bool done = false;
     const int r = try_skinny(fmt, count, descs, M, (cudaStream_t)stream, &done);
