@@ -27,7 +27,7 @@ def test_int3_quantize_bitexact(N, K):
     assert_bitexact(rows_np(c, s, z, "int3", N, K), (p, sb, zb), f"int3 quantise {N}x{K}")
 
 
-@pytest.mark.parametrize("M", [1, 2, 5, 17])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 17])
 @pytest.mark.parametrize("N,K", SHAPES)
 def test_int3_product_matches_oracle(M, N, K):
     W = _crafted_weights(N, K, seed=1400 + N)
