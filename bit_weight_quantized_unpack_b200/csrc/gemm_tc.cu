@@ -9,8 +9,8 @@
 //     D[n, m] = sum_k w_hat[n0 + n, k] * X[m0 + m, k]      (n < 128, m < BN)
 // and every dequantised weight is reused by all BN tokens of the tile.
 //
-// Warp roles (one persistent CTA of 16 warps per SM; tiles dealt to CTAs round robin), per
-// 64-wide k-block:
+// Warp roles (one persistent CTA of 16 warps per SM; tiles dealt to CTAs as tile_deal.cuh
+// describes), per 64-wide k-block:
 //   - warp 4 (one lane): TMA loads the activation tile [bn x 64] fp16 (128-byte swizzle) into
 //     an XSTAGES-deep ring, completing on xfull[s]; it waits xempty[s] before reusing a stage;
 //   - warps 8-15 (two teams of four warps, one weight row per thread, the teams taking
@@ -138,7 +138,7 @@ __device__ __forceinline__ TileInfo tile_info(const TcParamsT<CAP>& P, int tile,
 
 }  // namespace
 
-// Persistent: CTA b runs tiles b, b + gridDim.x, ... in order. Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31 = weight rows), 4 TMA producer,
+// Persistent: CTA b runs its dealt tiles (tile_deal.cuh) in increasing order. Warp roles: 0-3 epilogue (TMEM lanes 32w..32w+31 = weight rows), 4 TMA producer,
 // 5 MMA issuer (and TMEM owner), 8-15 dequantisers (two threads per weight row, 32 k each
 // per stage); 6-7 idle. The two 256-column TMEM accumulators let the epilogue of one tile
 // overlap the main loop of the next.
@@ -183,9 +183,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   tc::tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  // tiles are dealt to CTAs round robin (CTA b takes tiles b, b + gridDim.x, ...); the host
-  // orders each launch's matrices by tile cost, largest first, so every CTA gets the same mix
-  const int t_lo = blockIdx.x, t_step = gridDim.x, t_hi = P.total_tiles;
+  // this CTA's j-th tile (-1 past its last); the host orders each launch's matrices by tile
+  // cost, largest first, and chooses the dealing that evens out the CTAs' total cost
+  const TileDeal deal = P.deal;
+  const int ctas = gridDim.x, total = P.total_tiles, cta = blockIdx.x;
+  auto tile_of = [&](int j) { return dealt_tile(cta, j, ctas, total, deal); };
 
   bool timed_out = false;
   int it = 0;    // k-block sequence number over this CTA's tiles
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   if (warp == XPROD_WARP) {
     // activation tiles, one per k-block
     if (lane == 0) {
-      for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step) {
+      for (int j = 0, tile; (tile = tile_of(j)) >= 0 && !timed_out; ++j) {
         const TileInfo ti = tile_info(P, tile, mi);
         const TcMat& M = P.m[ti.mi];
         const uint32_t tx = (uint32_t)(ti.bn * BK * 2);
@@ -210,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
   } else if (warp == MMA_WARP) {
     if (lane == 0) {
       int lt = 0;
-      for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step, ++lt) {
+      for (int j = 0, tile; (tile = tile_of(j)) >= 0 && !timed_out; ++j, ++lt) {
         const TileInfo ti = tile_info(P, tile, mi);
         const int b = lt & 1;
         if (!tc::mbar_wait(bar_tempty + 8 * b, ((lt >> 1) & 1) ^ 1)) { timed_out = true; break; }
@@ -251,21 +253,22 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     };
     // A cursor over this CTA's (tile, k-block) sequence restricted to one team's k-blocks.
     struct Cursor {
-      int tile, kb, mi;
+      int j, tile, kb, mi;  // tile = this CTA's j-th tile, -1 past the last
       TileInfo ti;
     };
     auto cursor_start = [&](Cursor& c) {
-      c.tile = t_lo;
+      c.j = 0;
+      c.tile = tile_of(0);
       c.kb = team;
       c.mi = 0;
-      if (c.tile < t_hi) c.ti = tile_info(P, c.tile, c.mi);
+      if (c.tile >= 0) c.ti = tile_info(P, c.tile, c.mi);
     };
     auto cursor_next = [&](Cursor& c) {
       c.kb += 2;
       if (c.kb >= c.ti.nkb) {
         c.kb = team;
-        c.tile += t_step;
-        if (c.tile < t_hi) c.ti = tile_info(P, c.tile, c.mi);
+        c.tile = tile_of(++c.j);
+        if (c.tile >= 0) c.ti = tile_info(P, c.tile, c.mi);
       }
     };
     // Codes are not copied by TMA: a slow DRAM copy would hold up the activation copies
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     cursor_start(fc);
     int fseq = 0;
     auto fetch_next = [&]() {
-      if (fc.tile < t_hi) {
+      if (fc.tile >= 0) {
         const TcMat& Mf = P.m[fc.ti.mi];
         const int nf = min(fc.ti.n0 + r, Mf.N - 1);
         const uint8_t* src = reinterpret_cast<const uint8_t*>(Mf.codes) + (size_t)nf * (Mf.K / 2) + fc.kb * (BK / 2);
@@ -295,7 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     SzPair sz0{0, 0}, sz1{0, 0};
     auto sz_fetch = [&]() -> SzPair {
       SzPair v{0, 0};
-      if (sc.tile < t_hi) {
+      if (sc.tile >= 0) {
         const TcMat& Ms = P.m[sc.ti.mi];
         v = load_sz(Ms, min(sc.ti.n0 + r, Ms.N - 1), sc.kb >> 1);
         cursor_next(sc);
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     sz0 = sz_fetch();
     sz1 = sz_fetch();
     int cseq = 0;
-    for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step) {
+    for (int j = 0, tile; (tile = tile_of(j)) >= 0 && !timed_out; ++j) {
       const TileInfo ti = tile_info(P, tile, mi);
       for (int kb = team; kb < ti.nkb; kb += 2) {
         const int itk = it + kb;               // sequence number of this k-block
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_int4_kernel(const __grid_c
     int lt = 0, nst = 0;
     const uint32_t ebuf = sbase + OFF_E + (uint32_t)(warp * 2 * EPI_BYTES);
     uint16_t* ebuf_g = reinterpret_cast<uint16_t*>(smem + OFF_E + warp * 2 * EPI_BYTES);
-    for (int tile = t_lo; tile < t_hi && !timed_out; tile += t_step, ++lt) {
+    for (int j = 0, tile; (tile = tile_of(j)) >= 0 && !timed_out; ++j, ++lt) {
       const TileInfo ti = tile_info(P, tile, mi);
       const TcMat& M = P.m[ti.mi];
       const int b = lt & 1;
@@ -472,8 +475,25 @@ int tc_bn_for(int M) {
   return bn < XBN ? bn : XBN;
 }
 
+// The dealing of p's tiles to `grid` CTAs: the leading matrices whose tiles have the largest
+// cost against the cost of the next matrix's tiles (matrices come in non-increasing cost).
 template <int CAP>
-static cudaError_t launch_cap(const TcParamsT<CAP>& p, cudaStream_t stream) {
+static TileDeal deal_for(const TcParamsT<CAP>& p, int grid) {
+  const int c1 = p.m[0].tile_cost;
+  int n1 = 0, c2 = 0;
+  for (int i = 0; i < p.count; ++i) {
+    if (p.m[i].tile_cost != c1) {
+      c2 = p.m[i].tile_cost;
+      break;
+    }
+    n1 += p.m[i].tile_end - p.m[i].tile_begin;
+  }
+  if (c2 > c1) return TileDeal{0, 0, 0};  // not in cost order: plain round robin
+  return plan_deal(grid, n1, c1, c2);
+}
+
+template <int CAP>
+static cudaError_t launch_cap(TcParamsT<CAP>& p, cudaStream_t stream) {
   static std::atomic<uint64_t> attr{0};
   const int smem = SMEM_USED + 1024;  // + alignment slack
   cudaError_t e = ensure_smem_limit(gemm_tc_int4_kernel<CAP>, smem, attr);
@@ -481,11 +501,12 @@ static cudaError_t launch_cap(const TcParamsT<CAP>& p, cudaStream_t stream) {
   const int sms = device_sm_count();
   if (sms == 0) return cudaErrorInvalidDevice;
   const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+  p.deal = deal_for(p, grid);
   gemm_tc_int4_kernel<CAP><<<grid, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream) {
+cudaError_t launch_gemm_tc(TcParams& p, cudaStream_t stream) {
   if (p.count == 1) {
     TcParamsT<1> p1;
     p1.m[0] = p.m[0];

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "tile_deal.cuh"
+
 namespace wq {
 
 constexpr int kTcMaxBN = 256;   // tokens per tile (MMA N), also the TMEM columns allocated
@@ -35,13 +37,16 @@ struct TcParamsT {
   int64_t total_cost;
   int count;
   int total_tiles;
+  TileDeal deal;  // how the tiles are dealt to the CTAs (filled by launch_gemm_tc)
 };
 using TcParams = TcParamsT<kTcMaxMats>;
+static_assert(sizeof(TcParams) <= 32764, "kernel parameter block");
 
 bool tc_plan_mat(TcMat& t, const uint16_t* X, int M, const void* codes, const uint16_t* scale,
                  const uint16_t* zero, uint16_t* Y, int N, int K, int bn);
 int tc_bn_for(int M);
-cudaError_t launch_gemm_tc(const TcParams& p, cudaStream_t stream);
+// Fills p.deal for the grid it launches; p's matrices must be in non-increasing tile cost.
+cudaError_t launch_gemm_tc(TcParams& p, cudaStream_t stream);
 cudaError_t read_device_errors(unsigned int* flags, bool clear, cudaStream_t stream);
 // Device address of the error word on the current device (looked up once per device).
 unsigned int* device_error_word();
